@@ -1,0 +1,82 @@
+"""Plants plausible mistakes in the oracle (CPU only, via monkeypatch) and checks that at least one pin
+fails for each, so the pins are known to bite."""
+import numpy as np
+import pytest
+
+import importlib
+
+acc_mod = importlib.import_module("oracle.accept")
+bt_mod = importlib.import_module("oracle.build_tree")
+ta_mod = importlib.import_module("oracle.tree_attention")
+from tests import test_oracle_accept as TA
+from tests import test_oracle_attention as TT
+from tests import test_oracle_build as TB
+
+
+def fails(fn, *a):
+    try:
+        fn(*a)
+    except (AssertionError, ValueError, IndexError):
+        return True
+    return False
+
+
+def test_dropping_self_is_caught(monkeypatch):
+    def anc_no_self(parent):
+        anc = []
+        for i, p in enumerate(parent.tolist()):
+            base = (anc[p] | {p}) if p >= 0 else set()
+            anc.append(base)
+        return anc
+    monkeypatch.setattr(ta_mod, "ancestor_sets", anc_no_self)
+    assert fails(TT.test_star_equals_prefix_plus_self)
+
+
+def test_seeing_siblings_is_caught(monkeypatch):
+    orig = ta_mod.ancestor_sets
+
+    def anc_with_siblings(parent):
+        anc = orig(parent)
+        for i, p in enumerate(parent.tolist()):
+            anc[i] = anc[i] | {j for j in range(len(parent)) if parent[j] == p and p >= 0}
+        return anc
+    monkeypatch.setattr(ta_mod, "ancestor_sets", anc_with_siblings)
+    assert fails(TT.test_path_extraction_branch_factorisation, 4)
+
+
+def test_transposed_page_index_is_caught(monkeypatch):
+    def bad_gather(cache, block_row, slots, kv_head):
+        return cache[block_row[slots % 16 % len(block_row)], slots // 16 % 16, kv_head, :].astype(np.float64)
+    monkeypatch.setattr(ta_mod, "gather_slots", bad_gather)
+    assert fails(TT.test_chain_equals_causal_attention)
+
+
+def test_wrong_gqa_map_is_caught(monkeypatch):
+    orig = ta_mod.gather_slots
+    monkeypatch.setattr(ta_mod, "gather_slots", lambda c, r, s, h: orig(c, r, s, (h + 1) % c.shape[2]))
+    assert fails(TT.test_chain_equals_causal_attention)
+
+
+def test_wrong_depth_row_is_caught(monkeypatch):
+    orig = bt_mod.row_stats
+    calls = {"n": 0}
+
+    def shifted_stats(x):  # pretend the normaliser of each row were off by a depth-dependent amount
+        calls["n"] += 1
+        m, lse = orig(x)
+        return m, lse + 0.01 * calls["n"]
+    monkeypatch.setattr(bt_mod, "row_stats", shifted_stats)
+    assert fails(TB.test_brute_force_full_tree, 2, 3, 4, 40)
+
+
+def test_sibling_order_is_caught(monkeypatch):
+    monkeypatch.setattr(bt_mod, "topk_tokens", lambda x, k: np.argsort(np.asarray(x))[:k])
+    assert fails(TB.test_topk1_is_chain_of_argmaxes)
+
+
+def test_highest_id_tie_break_is_caught(monkeypatch):
+    def last_argmax(row):
+        row = np.asarray(row)
+        return len(row) - 1 - int(np.argmax(row[::-1]))
+    monkeypatch.setattr(acc_mod, "first_argmax", last_argmax)
+    assert fails(TA.test_argmax_ties_take_lowest_id)
