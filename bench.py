@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Benchmark of the tree-verify hot path on B200.
+
+One step = one pass of the whole hot path over one batch: jf_build_tree on the step's draft logits
+(best-first tree of `budget` nodes), jf_tree_attention of every tree node over the paged KV cache
+(prefix + the tree the step just built; Qwen3-8B attention shape by default), jf_accept of the built
+tree against the target logits.  Metric: tree nodes verified per second (whole job), with the
+attention kernel's achieved TFLOP/s and HBM GB/s against the measured B200 peaks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl jf|reference] [--workload qwen3_8b]
+
+N > 1 is launched with torchrun: every rank verifies its own independent batch (weak scaling, no
+collective on the data path); the step time is the max over ranks.  `--impl reference` times the CPU
+oracle (the deliberately slow, obviously correct float64 restatement of the method) on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # name: (batch, q heads, kv heads, prefix, budget, topk, max_depth, vocab, draft depths)
+    "qwen3_8b": dict(batch=1, hq=32, hkv=8, prefix=4096, budget=256, topk=4, max_depth=16, vocab=151936, depths=16),
+    "qwen3_30b_a3b": dict(batch=4, hq=32, hkv=4, prefix=32768, budget=256, topk=4, max_depth=16, vocab=151936,
+                          depths=16),
+    "serving": dict(batch=16, hq=32, hkv=8, prefix=4608, budget=64, topk=4, max_depth=12, vocab=151936, depths=16),
+}
+HEAD_DIM = 128
+PAGE = 16
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]), bf16_sus=float(d["bf16_tflops_sustained"]),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ----------------------------------------------------------------------------------------------
+# Inputs (seeded, synthetic; shapes of the pages' Qwen3 workloads)
+# ----------------------------------------------------------------------------------------------
+def make_inputs(cfg, seed):
+    from tree_verify_attention_jf_b200 import synth
+
+    B, N = cfg["batch"], cfg["budget"]
+    rng = np.random.default_rng(seed)
+    x, roots = synth.draft_logits(seed, B, cfg["depths"], cfg["vocab"])
+    prefix = [cfg["prefix"]] * B
+    pages_per_seq = [(P + N + PAGE - 1) // PAGE for P in prefix]
+    bt, num_pages = synth.page_pool(rng, pages_per_seq, interleave=True)
+    q = rng.standard_normal((B * N, cfg["hq"], HEAD_DIM), dtype=np.float32) * np.float32(0.5)
+    kv_shape = (num_pages, PAGE, cfg["hkv"], HEAD_DIM)
+    return dict(draft=x, roots=roots, q=q, kv_shape=kv_shape, block_table=bt, prefix=np.array(prefix, np.int32),
+                offsets=(np.arange(B + 1) * N).astype(np.int32))
+
+
+def visible_pairs(parent, prefix):
+    """sum over nodes of |visible set| = P + depth(node) (node with parent -1 has depth 1)."""
+    tot = 0
+    for b in range(parent.shape[0]):
+        d = np.zeros(parent.shape[1], dtype=np.int64)
+        for i in range(parent.shape[1]):
+            p = parent[b, i]
+            d[i] = 1 if p < 0 else d[p] + 1
+        tot += int(prefix[b]) * parent.shape[1] + int(d.sum())
+    return tot
+
+
+class ClockSampler:
+    def __init__(self, uuid, out_path):
+        self.proc = None
+        self.path = out_path
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.fh = open(out_path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={uuid if str(uuid).startswith('GPU-') else 'GPU-' + str(uuid)}", f"--query-gpu={q}", "--format=csv,noheader",
+                                          "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["unsampled"])
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1].split()[0]))
+                smax.append(float(f[2].split()[0]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["unsampled"])
+        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=max(smax), reasons=sorted(reasons), samples=len(sm))
+
+
+# ----------------------------------------------------------------------------------------------
+# CPU oracle leg (cpu_baseline and --impl reference)
+# ----------------------------------------------------------------------------------------------
+def oracle_step_rate(cfg, seed, budget_s=15.0, max_steps=40):
+    """Times the oracle over whole steps (build + attention + accept) of the same workload until about
+    `budget_s` seconds of CPU work; returns (nodes/s, steps timed, threads)."""
+    from oracle.accept import accept as o_accept
+    from oracle.build_tree import build_tree as o_build
+    from oracle.tree_attention import tree_attention
+    from tree_verify_attention_jf_b200 import synth
+
+    inp = make_inputs(cfg, seed)
+    B, N = cfg["batch"], cfg["budget"]
+    rng = np.random.default_rng(seed + 1)
+    k = synth.bf16_round(rng.standard_normal(inp["kv_shape"], dtype=np.float32) * np.float32(0.5))
+    v = synth.bf16_round(rng.standard_normal(inp["kv_shape"], dtype=np.float32) * np.float32(0.5))
+    q = synth.bf16_round(inp["q"])
+    tree = o_build(inp["draft"], inp["roots"], cfg["topk"], N, cfg["max_depth"])
+    tgt, _ = synth.target_logits_with_path(seed + 2, tree["parent"], tree["token"], cfg["vocab"])
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        tree = o_build(inp["draft"], inp["roots"], cfg["topk"], N, cfg["max_depth"])
+        tree_attention(q, k, v, inp["block_table"], inp["prefix"], inp["offsets"], tree["parent"].reshape(-1),
+                       1.0 / np.sqrt(HEAD_DIM), cfg["hkv"])
+        o_accept(tree["token"], tree["parent"], tgt, cfg["max_depth"])
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or steps >= max_steps:
+            break
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    return B * N * steps / el, steps, el, threads
+
+
+# ----------------------------------------------------------------------------------------------
+# GPU leg
+# ----------------------------------------------------------------------------------------------
+def run_gpu(args, cfg, rank, world, device):
+    import torch
+
+    from tree_verify_attention_jf_b200 import api, synth
+
+    torch.cuda.set_device(device)
+    seed = 1000 + rank
+    inp = make_inputs(cfg, seed)
+    B, N, V = cfg["batch"], cfg["budget"], cfg["vocab"]
+    gen = torch.Generator(device=device).manual_seed(seed)
+    kc = (torch.randn(inp["kv_shape"], generator=gen, device=device) * 0.5).to(torch.bfloat16)
+    vc = (torch.randn(inp["kv_shape"], generator=gen, device=device) * 0.5).to(torch.bfloat16)
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+    draft_h = torch.from_numpy(inp["draft"]).pin_memory()
+    roots = i32(inp["roots"])
+    q_h = torch.from_numpy(inp["q"]).to(torch.bfloat16).pin_memory()
+    draft = draft_h.to(device)
+    q = q_h.to(device)
+    bt, prefix, offs = i32(inp["block_table"]), i32(inp["prefix"]), i32(inp["offsets"])
+    out = torch.empty_like(q)
+    ws_attn = api.AttentionWorkspace(torch.device(device))
+    ws_build = api.build_tree_workspace(B, cfg["depths"], V, cfg["topk"], device)
+    tree = api.build_tree(draft, roots, cfg["topk"], N, cfg["max_depth"], workspace=ws_build)
+    torch.cuda.synchronize()
+    par_h, tok_h = tree["parent"].cpu().numpy(), tree["token"].cpu().numpy()
+    # Target logits that agree with this tree along a seeded path (the tree is fixed by the seeded draft
+    # logits; it is read back once, outside any timed region, only to plant the path).
+    tgt_np, paths = synth.target_logits_with_path(seed + 2, par_h, tok_h, V)
+    tgt_h = torch.from_numpy(tgt_np).pin_memory()
+    tgt = tgt_h.to(device)
+    del tgt_np
+    acc_out = dict(accepted_len=torch.empty(B, dtype=torch.int32, device=device),
+                   path=torch.empty(B, cfg["max_depth"] + 1, dtype=torch.int32, device=device),
+                   bonus=torch.empty(B, dtype=torch.int32, device=device))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        api.build_tree(draft, roots, cfg["topk"], N, cfg["max_depth"], workspace=ws_build, out=tree)
+        ev[1].record(stream)
+        api.tree_attention(q, kc, vc, bt, prefix, offs, tree["parent"].view(-1), 1.0 / np.sqrt(HEAD_DIM), out=out,
+                           workspace=ws_attn)
+        ev[2].record(stream)
+        api.accept(tree["token"], tree["parent"], tgt, cfg["max_depth"], out=acc_out)
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for _ in range(args.warmup):
+        ev[0].record(stream)
+        step()
+        ev[3].record(stream)
+    torch.cuda.synchronize()
+    expect_len = [len(p) - 1 for p in paths]
+    got_len = acc_out["accepted_len"].cpu().tolist()
+    if got_len != expect_len:
+        raise RuntimeError(f"accepted lengths {got_len} != planted {expect_len}")
+
+    # ---- timed region: K steps, per-step events, L2 flushed between steps (outside the events)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.get_device_properties(device).uuid, os.path.join(ROOT, "gpurun_out",
+                                                                                        f"clocks_r{rank}.csv")) \
+        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(
+            torch.cuda.get_device_properties(device).uuid, f"/tmp/jf_clocks_r{rank}.csv")
+    time.sleep(0.3)
+    step_ms, attn_ms, build_ms, accept_ms = [], [], [], []
+    for _ in range(args.steps):
+        flush.zero_()
+        ev[0].record(stream)
+        step()
+        ev[3].record(stream)
+        ev[3].synchronize()
+        step_ms.append(ev[0].elapsed_time(ev[3]))
+        build_ms.append(ev[0].elapsed_time(ev[1]))
+        attn_ms.append(ev[1].elapsed_time(ev[2]))
+        accept_ms.append(ev[2].elapsed_time(ev[3]))
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+
+    # ---- e2e: the same step through the public API with host buffers; H2D of the step's inputs
+    # (draft logits, tree queries, target logits) from pinned memory and D2H of its result inside
+    res_h = torch.empty(B * (cfg["max_depth"] + 3), dtype=torch.int32).pin_memory()
+    e2e_ms = []
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, min(args.steps, 20))
+    for _ in range(n_e2e):
+        flush.zero_()
+        e_s.record(stream)
+        draft.copy_(draft_h, non_blocking=True)
+        q.copy_(q_h, non_blocking=True)
+        tgt.copy_(tgt_h, non_blocking=True)
+        step()
+        res = torch.cat([acc_out["accepted_len"], acc_out["bonus"], acc_out["path"].view(-1)])
+        res_h.copy_(res, non_blocking=True)
+        e_e.record(stream)
+        e_e.synchronize()
+        e2e_ms.append(e_s.elapsed_time(e_e))
+    h2d = draft_h.numel() * 4 + q_h.numel() * 2 + tgt_h.numel() * 4
+    d2h = res_h.numel() * 4
+    return dict(step_ms=step_ms, attn_ms=attn_ms, build_ms=build_ms, accept_ms=accept_ms, clocks=clocks,
+                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, parent=par_h)
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="jf", choices=["jf", "reference"])
+    ap.add_argument("--workload", default="qwen3_8b", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    metric = "tree nodes verified/sec"
+    config = {"workload": f"{args.workload}_tree_verify", "batch": cfg["batch"], "q_heads": cfg["hq"],
+              "kv_heads": cfg["hkv"], "head_dim": HEAD_DIM, "prefix": cfg["prefix"], "page_size": PAGE,
+              "budget": cfg["budget"], "topk": cfg["topk"], "max_depth": cfg["max_depth"], "vocab": cfg["vocab"],
+              "step": "build_tree + tree_attention (one layer) + accept", "parallelism": f"replicas{world}",
+              "l2": "flushed between steps (256 MiB write outside the timed events)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        rate, steps, el, threads = oracle_step_rate(cfg, 1000)
+        line = {"impl": "reference", "metric": metric, "value": rate, "unit": "nodes/s", "n_gpus": args.gpus,
+                "steps": steps, "warmup": 0, "ms_per_step": 1e3 * el / steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+                "config": config,
+                "cpu_baseline": {"value": rate, "unit": "nodes/s", "cores": threads, "kind": "oracle",
+                                 "sample": f"{steps} whole step(s) of the workload, {el:.1f} s"},
+                "e2e": {"value": rate, "unit": "nodes/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = f"cuda:{local}"
+    r = run_gpu(args, cfg, rank, world, device)
+    mean_step = statistics.mean(r["step_ms"])
+    step_ms = max_over_ranks(mean_step, world, device)
+    e2e_step = max_over_ranks(statistics.mean(r["e2e_ms"]), world, device)
+    attn_ms = statistics.mean(r["attn_ms"])
+    B, N = cfg["batch"], cfg["budget"]
+    nodes = B * N * world
+    pk = peaks()
+    pairs = visible_pairs(r["parent"], [cfg["prefix"]] * B)
+    flops = 4.0 * HEAD_DIM * cfg["hq"] * pairs
+    kv_bytes = B * cfg["hkv"] * (cfg["prefix"] + N) * HEAD_DIM * 2 * 2
+    qo_bytes = 2 * B * N * cfg["hq"] * HEAD_DIM * 2
+    meta_bytes = B * (4 * (cfg["prefix"] + N + PAGE - 1) // PAGE + 4 * N + 12)
+    tflops = flops / (attn_ms * 1e-3) / 1e12
+    gbs = (kv_bytes + qo_bytes + meta_bytes) / (attn_ms * 1e-3) / 1e9
+    shares = {"build_tree": statistics.mean(r["build_ms"]) / mean_step,
+              "tree_attention": attn_ms / mean_step, "accept": statistics.mean(r["accept_ms"]) / mean_step}
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        rate, steps, el, threads = oracle_step_rate(cfg, 1000)
+        cpu = {"value": rate, "unit": "nodes/s", "cores": threads, "kind": "oracle",
+               "sample": f"{steps} whole step(s) of the same workload (build + attention + accept), {el:.1f} s"}
+    line = {
+        "metric": metric, "value": nodes / (step_ms * 1e-3), "unit": "nodes/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)", "config": config,
+        "roofline": {"kernel": "jf::attn::tree_attention_kernel", "bound": "tensor", "achieved": tflops,
+                     "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops / pk["bf16"], "traffic": None,
+                     "peak_source": pk["src"] + " bf16 burst",
+                     "hbm_achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm"],
+                     "algorithmic_flops": flops, "algorithmic_bytes": kv_bytes + qo_bytes + meta_bytes},
+        "kernel_ms": {"build_tree": statistics.mean(r["build_ms"]), "tree_attention": attn_ms,
+                      "accept": statistics.mean(r["accept_ms"])},
+        "time_share": shares,
+        "e2e": {"value": nodes / (e2e_step * 1e-3), "unit": "nodes/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": 4 * args.steps,
+        "clocks": r["clocks"],
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

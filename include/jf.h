@@ -1,0 +1,167 @@
+/*
+ * jf.h -- C ABI of libjf.so: the tree-verify hot path of causal parallel tree drafting
+ * (JetFlow / JetSpec) on NVIDIA B200 (sm_100a).
+ *
+ * Sources (page titles; the pages print no code and define no API):
+ *   [JF] "JetFlow: Breaking the Scaling Ceiling of Speculative Decoding with Parallel Tree Drafting",
+ *        technical summary: section 1 (verification and acceptance), section 2 (tree-causal attention
+ *        mask, branch factorisation, best-first tree construction to a budget), section 3 (paged
+ *        attention inside a serving engine), section 4 (budgets 16..256, tau accepted tokens).
+ *   [JS] "JetSpec" paper page, abstract.
+ *
+ * Conventions shared by every call
+ *   - Every array argument is DEVICE memory owned by the caller; the library never allocates,
+ *     frees or retains a pointer after the call returns.  Scratch space is passed in as
+ *     `workspace`, sized by the matching *_workspace_size() query.
+ *   - Calls are asynchronous and stream-ordered on `stream` (0 = legacy default stream).  No call
+ *     synchronises the host.  Calls on different streams may run concurrently as long as they use
+ *     different workspaces and outputs.
+ *   - Problems that the host can see (null pointers, unsupported shapes, short workspace,
+ *     misaligned pointers) return an error code synchronously and launch nothing.
+ *   - Problems that depend on device data (a parent index out of range, a page id out of range,
+ *     a sequence longer than its block table, malformed tree_offsets) are detected on the device:
+ *     the first such code is written with atomicCAS into `*dev_status` (an int32 the caller zeroes
+ *     before the call), and the outputs of the offending sequence are left unwritten.  The device
+ *     never traps.  `dev_status` may be NULL, in which case device-detected problems are silent.
+ *   - Every device-side wait is bounded; if one runs out (it never should) the kernel writes
+ *     JF_ERR_TIMEOUT to `*dev_status` and returns.
+ *   - bf16 arrays are passed as `const void*`: IEEE-754 bfloat16, 2 bytes per element.
+ */
+#ifndef JF_H_
+#define JF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define JF_API __attribute__((visibility("default")))
+#else
+#define JF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* jf_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  JF_OK = 0,
+  JF_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misaligned pointer, short workspace */
+  JF_ERR_UNSUPPORTED = 2,  /* head_dim != 128, page_size != 16, bad GQA ratio, sizes above limits */
+  JF_ERR_CUDA = 3,         /* a CUDA runtime / driver call failed (launch, attribute, tensor map) */
+  JF_ERR_DEVICE_CHECK = 4, /* device-side data check failed (written to *dev_status only) */
+  JF_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out (written to *dev_status only) */
+} jf_status;
+
+/* Human-readable name of a status code.  Never NULL. */
+JF_API const char* jf_status_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+JF_API int jf_version(void);
+
+/* ------------------------------------------------------------------------------------------
+ * jf_tree_attention -- tree-causal attention of every draft-tree node over the paged KV cache.
+ *
+ * Defines [JF section 2, "tree-causal attention mask"; branch factorisation
+ * q(pi(v)|x) = prod_{u in pi(v)} q(y_u | x, h_x, pi_<u)]: the query of tree node n of sequence b
+ * attends to all prefix_lens[b] cached prefix tokens and to the tree slots of its own ancestors
+ * and itself, never to descendants or unrelated siblings.  For q head h (kv head h / (Hq/Hkv)):
+ *     s_t  = sm_scale * <q[n,h,:], K[t]>               for visible logical slots t
+ *     out  = sum_t softmax(s)_t V[t]                    (bf16, round-to-nearest-even)
+ *     lse  = ln sum_t exp(s_t)                          (fp32, optional)
+ * Visible slots of node n (local index within its sequence): t in [0, P) and t = P + j for every
+ * j on n's root path (j = n, parent[n], parent[parent[n]], ... until -1).
+ *
+ * Layouts (row-major, innermost last):
+ *   q            bf16  [total_nodes, num_q_heads, head_dim]; sequence b owns rows
+ *                      [tree_offsets[b], tree_offsets[b+1])
+ *   k_cache,
+ *   v_cache      bf16  [num_pages, page_size, num_kv_heads, head_dim]
+ *   block_table  int32 [batch, max_pages_per_seq]: logical page p of sequence b is physical page
+ *                      block_table[b*max_pages_per_seq + p]; logical slot t is row t % page_size of
+ *                      logical page t / page_size.  The tree nodes' K/V must already sit at logical
+ *                      slots prefix_lens[b] .. prefix_lens[b] + N_b - 1 (node order).
+ *   prefix_lens  int32 [batch], >= 0
+ *   tree_offsets int32 [batch+1], tree_offsets[0] = 0, non-decreasing, tree_offsets[batch] =
+ *                      total_nodes; N_b = tree_offsets[b+1] - tree_offsets[b] <= 256
+ *   parent       int32 [total_nodes], local index of the parent within the sequence, in
+ *                      [-1, i-1] for node i (-1 = child of the cached prefix)
+ *   out          bf16  [total_nodes, num_q_heads, head_dim]
+ *   lse          fp32  [total_nodes, num_q_heads] or NULL
+ * Supported: head_dim == 128, page_size == 16, num_q_heads % num_kv_heads == 0 with
+ * Hq/Hkv in {1, 2, 4, 8, 16}, batch <= 2048.  q, k_cache, v_cache and out must be 16-byte aligned.
+ * Cache slots beyond prefix_lens[b] + N_b in the last used page are never part of the result.
+ *
+ * workspace: at least jf_tree_attention_workspace_size(...) bytes of device memory, 256-byte
+ * aligned, zero-filled before its FIRST use with this library; every call that completes leaves it
+ * zeroed again where it needs zeros, so it can be reused across calls without a memset.
+ * ------------------------------------------------------------------------------------------ */
+JF_API size_t jf_tree_attention_workspace_size(int batch, int num_q_heads, int num_kv_heads, int total_nodes);
+
+JF_API jf_status jf_tree_attention(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_table, int max_pages_per_seq,
+                            const int32_t* prefix_lens, const int32_t* tree_offsets,
+                            const int32_t* parent, int batch, int total_nodes, int num_q_heads,
+                            int num_kv_heads, int head_dim, int page_size, int num_pages,
+                            float sm_scale, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, jf_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * jf_build_tree -- best-first draft-tree construction under a token budget.
+ *
+ * Defines [JF section 2, "tree construction": the head emits logits for all depths in parallel; the
+ * branch score is the cumulative draft log-probability; best-first expansion up to a budget such
+ * as 256].  Reading of the per-depth input: row d-1 of draft_logits scores every child at depth d,
+ * so all depth-(d-1) nodes share the same top-k children.  Steps:
+ *   1. per (b, d): lse_d = m + ln sum_v exp(x_v - m) with m = max_v x_v (float64 accumulation and
+ *      float64 exp), the top-k tokens by (logit descending, token id ascending), and
+ *      lp[d][r] = x_tok - lse_d in float64;
+ *   2. node 0 = root_tokens[b], parent -1, depth 0, score 0; the budget counts the root;
+ *   3. candidates (p, r) with key score(p) + lp[depth(p)+1][r] are popped best-first by
+ *      (key descending, depth ascending, parent index ascending, rank ascending); the popped
+ *      candidate becomes the next node (parent p, token = r-th top token of its depth, score = key
+ *      rounded to fp32); its sibling (p, r+1) and its first child (i, 0) (if depth < max_depth) join
+ *      the queue; repeat until `budget` nodes exist.
+ * The output order is pop order, so parent[i] < i.
+ *
+ * Layouts: draft_logits fp32 [batch, depths, vocab]; root_tokens int32 [batch];
+ *          parent, token int32 [batch, budget]; score fp32 [batch, budget]; depth int32
+ *          [batch, budget] or NULL.
+ * Limits: 1 <= topk <= 8, topk <= vocab, 1 <= max_depth <= depths <= 64, 1 <= budget <= 1024 and
+ *         budget <= 1 + sum_{d=1..max_depth} topk^d, vocab < 2^31.
+ * workspace: jf_build_tree_workspace_size(...) bytes (no zero-fill needed).
+ * ------------------------------------------------------------------------------------------ */
+JF_API size_t jf_build_tree_workspace_size(int batch, int depths, int vocab, int topk);
+
+JF_API jf_status jf_build_tree(const float* draft_logits, const int32_t* root_tokens, int batch, int depths,
+                        int vocab, int topk, int budget, int max_depth, int32_t* parent,
+                        int32_t* token, float* score, int32_t* depth, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, jf_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * jf_accept -- greedy acceptance walk over the verified tree.
+ *
+ * Defines [JF section 1: the target verifies the drafted tokens in parallel and keeps the longest
+ * agreeing prefix; section 4: tau accepted tokens]: cur = 0 (root), L = 0; loop:
+ * a = argmax_v target_logits[b, cur, v] (lowest id on ties); stop if L == max_depth; otherwise look
+ * for a child c of cur (parent[c] == cur) with token[c] == a (lowest c if several); if found,
+ * L += 1, path[L] = c, cur = c, repeat; else stop.  bonus_token = a from the last iteration.
+ *
+ * Layouts: token, parent int32 [batch, num_nodes] (node 0 is the root, parent[0] = -1,
+ *          parent[i] in [-1, i-1]); target_logits fp32 [batch, num_nodes, vocab], row i = the
+ *          target's next-token logits after node i; accepted_len int32 [batch] (root excluded,
+ *          0..max_depth); path int32 [batch, max_depth+1] (path[0] = 0, unused entries -1);
+ *          bonus_token int32 [batch].
+ * Limits: 1 <= num_nodes <= 1024, 0 <= max_depth <= 1023, 1 <= vocab < 2^31.  target_logits must
+ *         be 16-byte aligned; NaN logits give an unspecified (but in-range) argmax.
+ * ------------------------------------------------------------------------------------------ */
+JF_API jf_status jf_accept(const int32_t* token, const int32_t* parent, const float* target_logits,
+                    int batch, int num_nodes, int vocab, int max_depth, int32_t* accepted_len,
+                    int32_t* path, int32_t* bonus_token, int32_t* dev_status, jf_stream_t stream);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* JF_H_ */

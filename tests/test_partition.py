@@ -1,0 +1,81 @@
+"""Host-side model of the attention kernel's stream-K partition (the same integer formulas as the
+device plan): every (unit, kv tile) pair is covered exactly once, a unit's sharing CTAs are exactly
+those whose range intersects it, partial slots never collide, and every CTA's range is non-empty."""
+import itertools
+
+import numpy as np
+import pytest
+
+BN, BM = 128, 128
+
+
+def plan(prefix, nodes, hkv, group):
+    work = []
+    for P, N in zip(prefix, nodes):
+        if N == 0:
+            work.append(0)
+            continue
+        kt = (P + N + BN - 1) // BN
+        mt = (N * group + BM - 1) // BM
+        work.append(hkv * mt * kt)
+    cum = np.concatenate([[0], np.cumsum(work)]).astype(np.int64)
+    return cum
+
+
+def segments(prefix, nodes, hkv, group, grid):
+    cum = plan(prefix, nodes, hkv, group)
+    W = int(cum[-1])
+    G = min(grid, W)
+    cta_of = lambda x: ((x + 1) * G - 1) // W
+    out = []
+    for c in range(G):
+        x, xend = c * W // G, (c + 1) * W // G
+        assert xend > x
+        b = 0
+        while x < xend:
+            while cum[b + 1] <= x:
+                b += 1
+            P, N = prefix[b], nodes[b]
+            kt = (P + N + BN - 1) // BN
+            mtn = (N * group + BM - 1) // BM
+            local = x - cum[b]
+            unit = local // kt
+            kb = local - unit * kt
+            u0, u1 = cum[b] + unit * kt, cum[b] + unit * kt + kt
+            e = min(xend, u1)
+            c0, c1 = cta_of(u0), cta_of(u1 - 1)
+            slot = 2 * c + 1 if c == c0 else 2 * c
+            out.append(dict(cta=c, b=b, kvh=unit // mtn, mt=unit % mtn, kb=kb, ke=kb + (e - x), c0=c0, c1=c1, slot=slot))
+            x = e
+    return out, W, G
+
+
+@pytest.mark.parametrize("prefix,nodes,hkv,group,grid", [
+    ([256], [16], 1, 4, 148),
+    ([4096], [256], 8, 4, 148),
+    ([32768] * 4, [256] * 4, 4, 8, 148),
+    (list(np.random.default_rng(0).integers(1024, 8193, 16)), [64] * 16, 8, 4, 148),
+    ([0, 5, 300, 17], [3, 0, 256, 1], 2, 2, 7),
+    ([10] * 50, [1] * 50, 1, 1, 148),
+])
+def test_cover_exactly_once(prefix, nodes, hkv, group, grid):
+    segs, W, G = segments(prefix, nodes, hkv, group, grid)
+    seen = {}
+    for s in segs:
+        for t in range(s["kb"], s["ke"]):
+            key = (s["b"], s["kvh"], s["mt"], t)
+            assert key not in seen
+            seen[key] = s["cta"]
+    assert len(seen) == W
+    units = {}
+    for s in segs:
+        units.setdefault((s["b"], s["kvh"], s["mt"]), []).append(s)
+    slots = set()
+    for u, ss in units.items():
+        ctas = sorted(x["cta"] for x in ss)
+        assert ctas == list(range(ss[0]["c0"], ss[0]["c1"] + 1))
+        if len(ss) > 1:
+            for x in ss:
+                assert x["slot"] not in slots
+                slots.add(x["slot"])
+                assert x["slot"] < 2 * G

@@ -1,0 +1,128 @@
+"""Torch-facing calls of the tree-verify hot path.  PyTorch only supplies device memory and the stream;
+each function checks dtypes/shapes/devices, passes raw pointers to libjf.so (:mod:`._lib`) and returns.
+Nothing here computes any part of the method."""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+PAGE_SIZE = 16
+HEAD_DIM = 128
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, device: torch.device) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} must live on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class AttentionWorkspace:
+    """Zero-initialised scratch for :func:`tree_attention` (split-KV partials and per-row counters).
+    One per stream; reusable across calls (every completed call leaves it zeroed where needed)."""
+
+    def __init__(self, device: torch.device):
+        n = _lib.lib().jf_tree_attention_workspace_size(0, 0, 0, 0)
+        self.buf = torch.zeros(n, dtype=torch.uint8, device=device)
+
+    @property
+    def nbytes(self) -> int:
+        return self.buf.numel()
+
+
+def tree_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor,
+                   prefix_lens: torch.Tensor, tree_offsets: torch.Tensor, parent: torch.Tensor, sm_scale: float,
+                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                   workspace: Optional[AttentionWorkspace] = None, dev_status: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """jf_tree_attention: q bf16 [T, Hq, 128]; k/v_cache bf16 [pages, 16, Hkv, 128]; block_table int32
+    [B, max_pages]; prefix_lens int32 [B]; tree_offsets int32 [B+1]; parent int32 [T].  Returns out."""
+    dev = q.device
+    T, Hq, D = q.shape
+    num_pages, page, Hkv, D2 = k_cache.shape
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, dev)
+    _need(v_cache, "v_cache", torch.bfloat16, dev)
+    for name, t in (("block_table", block_table), ("prefix_lens", prefix_lens), ("tree_offsets", tree_offsets),
+                    ("parent", parent)):
+        _need(t, name, torch.int32, dev)
+    if v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache shapes differ")
+    B = prefix_lens.numel()
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev)
+    if workspace is None:
+        workspace = AttentionWorkspace(dev)
+    code = _lib.lib().jf_tree_attention(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1] if block_table.dim() == 2 else 0,
+        _ptr(prefix_lens), _ptr(tree_offsets), _ptr(parent), B, T, Hq, Hkv, D, page, num_pages, float(sm_scale),
+        _ptr(out), _ptr(lse), _ptr(workspace.buf), workspace.nbytes, _ptr(dev_status), _stream(stream))
+    _lib.check("jf_tree_attention", code)
+    return out
+
+
+def build_tree_workspace(batch: int, depths: int, vocab: int, topk: int, device) -> torch.Tensor:
+    n = _lib.lib().jf_build_tree_workspace_size(batch, depths, vocab, topk)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def build_tree(draft_logits: torch.Tensor, root_tokens: torch.Tensor, topk: int, budget: int, max_depth: int,
+               workspace: Optional[torch.Tensor] = None, out: Optional[dict] = None,
+               dev_status: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """jf_build_tree: draft_logits fp32 [B, depths, V], root_tokens int32 [B] -> dict of parent, token,
+    depth (int32 [B, budget]) and score (fp32 [B, budget])."""
+    dev = draft_logits.device
+    B, depths, V = draft_logits.shape
+    _need(draft_logits, "draft_logits", torch.float32, dev)
+    _need(root_tokens, "root_tokens", torch.int32, dev)
+    if out is None:
+        out = dict(parent=torch.empty(B, budget, dtype=torch.int32, device=dev),
+                   token=torch.empty(B, budget, dtype=torch.int32, device=dev),
+                   score=torch.empty(B, budget, dtype=torch.float32, device=dev),
+                   depth=torch.empty(B, budget, dtype=torch.int32, device=dev))
+    if workspace is None:
+        workspace = build_tree_workspace(B, depths, V, topk, dev)
+    code = _lib.lib().jf_build_tree(
+        _ptr(draft_logits), _ptr(root_tokens), B, depths, V, topk, budget, max_depth, _ptr(out["parent"]),
+        _ptr(out["token"]), _ptr(out["score"]), _ptr(out.get("depth")), _ptr(workspace), workspace.numel(),
+        _ptr(dev_status), _stream(stream))
+    _lib.check("jf_build_tree", code)
+    return out
+
+
+def accept(token: torch.Tensor, parent: torch.Tensor, target_logits: torch.Tensor, max_depth: int,
+           out: Optional[dict] = None, dev_status: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """jf_accept: token, parent int32 [B, N]; target_logits fp32 [B, N, V] -> dict of accepted_len int32 [B],
+    path int32 [B, max_depth + 1], bonus int32 [B]."""
+    dev = target_logits.device
+    B, N, V = target_logits.shape
+    _need(token, "token", torch.int32, dev)
+    _need(parent, "parent", torch.int32, dev)
+    _need(target_logits, "target_logits", torch.float32, dev)
+    if out is None:
+        out = dict(accepted_len=torch.empty(B, dtype=torch.int32, device=dev),
+                   path=torch.empty(B, max_depth + 1, dtype=torch.int32, device=dev),
+                   bonus=torch.empty(B, dtype=torch.int32, device=dev))
+    code = _lib.lib().jf_accept(_ptr(token), _ptr(parent), _ptr(target_logits), B, N, V, max_depth,
+                                _ptr(out["accepted_len"]), _ptr(out["path"]), _ptr(out["bonus"]), _ptr(dev_status),
+                                _stream(stream))
+    _lib.check("jf_accept", code)
+    return out

@@ -1,0 +1,257 @@
+// accept.cu -- greedy acceptance walk over the verified draft tree (sm_100a, SIMT + clusters).
+//
+// What it computes ("JetFlow: Breaking the Scaling Ceiling of Speculative Decoding with Parallel Tree
+// Drafting", technical summary section 1 and section 4): starting at the root, repeatedly take the
+// target model's argmax at the current node and move to the child carrying that token; the walk's
+// length is the number of accepted draft tokens (tau), the last argmax is the bonus token.
+//
+// Design: the walk is a chain of dependent argmaxes over 151936-entry rows, so latency matters more
+// than bandwidth.  Each sequence gets one thread-block cluster (16 CTAs where the GPU allows it,
+// else 8); every CTA reduces its slice of the current row with 16-byte loads issued eight deep, the
+// partial (value, id) pairs are exchanged through distributed shared memory, and every CTA derives
+// the same next node.  While a row is being reduced, the rows of the
+// current node's children (the only candidates for the next step) are prefetched into L2 with bulk
+// prefetches, so the next step reads from L2.
+#include <cooperative_groups.h>
+
+#include "jf_device.cuh"
+#include "jf_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace jf {
+namespace acc {
+
+constexpr int kMaxCluster = 16;
+constexpr int kThreads = 512;
+constexpr int kUnroll = 8;
+
+struct Best {
+  float v;
+  int id;
+};
+
+__device__ __forceinline__ bool better(float v, int id, float bv, int bid) {
+  return v > bv || (v == bv && id < bid);
+}
+
+__device__ __forceinline__ void take(float v, int id, float& bv, int& bid) {
+  if (better(v, id, bv, bid)) {
+    bv = v;
+    bid = id;
+  }
+}
+
+__device__ __forceinline__ void prefetch_l2(const float* p, long long n) {
+  // prefetch the 16-byte aligned interior of [p, p + n)
+  uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  uintptr_t e = reinterpret_cast<uintptr_t>(p + n);
+  a = (a + 15) & ~static_cast<uintptr_t>(15);
+  e &= ~static_cast<uintptr_t>(15);
+  while (a < e) {
+    const uintptr_t len = (e - a) > (1u << 20) ? (1u << 20) : (e - a);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(static_cast<uint32_t>(len)) : "memory");
+    a += len;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+    accept_kernel(const int32_t* __restrict__ token, const int32_t* __restrict__ parent,
+                  const float* __restrict__ logits, int num_nodes, int vocab, int max_depth,
+                  int32_t* __restrict__ accepted_len, int32_t* __restrict__ path, int32_t* __restrict__ bonus,
+                  int32_t* __restrict__ status) {
+  __shared__ int s_tok[kMaxAcceptNodes];
+  __shared__ int s_par[kMaxAcceptNodes];
+  __shared__ int s_path[kMaxAcceptNodes + 1];
+  __shared__ Best s_slot[2];  // this CTA's partial argmax, double-buffered across steps
+  __shared__ Best s_warp[kThreads / 32];
+  __shared__ int s_kids[kMaxAcceptNodes];
+  __shared__ int s_nkids, s_match, s_arg, s_bad;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int b = blockIdx.x / C;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t* tk = token + static_cast<long long>(b) * num_nodes;
+  const int32_t* pr = parent + static_cast<long long>(b) * num_nodes;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  for (int i = tid; i < num_nodes; i += kThreads) {
+    const int pi = pr[i];
+    s_par[i] = pi;
+    s_tok[i] = tk[i];
+    if (pi < -1 || pi >= i) s_bad = 1;
+  }
+  __syncthreads();
+  if (s_bad) {  // every CTA of the cluster sees the same data and leaves here together
+    if (rank == 0 && tid == 0) report(status, JF_ERR_DEVICE_CHECK);
+    return;
+  }
+  // this CTA's slice of every row (a multiple of 4 entries, so 16-byte loads stay aligned)
+  const int per = ((vocab + C - 1) / C + 3) & ~3;
+  const int lo = min(vocab, rank * per);
+  const int hi = min(vocab, lo + per);
+  const float* rows = logits + static_cast<long long>(b) * num_nodes * vocab;
+  const bool vec = (vocab % 4) == 0;  // rows then start 16-byte aligned (the base is checked on the host)
+
+  int cur = 0, L = 0, a = 0;
+  if (tid == 0) s_path[0] = 0;
+  for (int step = 0;; ++step) {
+    const float* row = rows + static_cast<long long>(cur) * vocab;
+    // children of cur: the candidates for the next row; prefetch their slices into L2
+    if (tid == 0) {
+      s_nkids = 0;
+      s_match = INT_MAX;
+    }
+    __syncthreads();
+    for (int c = tid; c < num_nodes; c += kThreads) {
+      if (s_par[c] == cur) s_kids[atomicAdd(&s_nkids, 1)] = c;
+    }
+    __syncthreads();
+    const int nk = s_nkids;
+    if (L < max_depth && tid < nk && hi > lo) {
+      prefetch_l2(rows + static_cast<long long>(s_kids[tid]) * vocab + lo, hi - lo);
+    }
+    // argmax of row cur over [lo, hi): lowest id among equal maxima
+    float bv = -INFINITY;
+    int bid = INT_MAX;
+    if (vec) {
+      const float4* row4 = reinterpret_cast<const float4*>(row);
+      const int lo4 = lo >> 2, hi4 = hi >> 2;
+      for (int base = lo4 + tid; base < hi4; base += kUnroll * kThreads) {
+        float4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int idx = base + u * kThreads;
+          v[u] = idx < hi4 ? __ldcg(row4 + idx) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int i0 = (base + u * kThreads) * 4;
+          take(v[u].x, i0, bv, bid);
+          take(v[u].y, i0 + 1, bv, bid);
+          take(v[u].z, i0 + 2, bv, bid);
+          take(v[u].w, i0 + 3, bv, bid);
+        }
+      }
+    } else {
+      for (int base = lo + tid; base < hi; base += kUnroll * kThreads) {
+        float v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int idx = base + u * kThreads;
+          v[u] = idx < hi ? __ldcg(row + idx) : -INFINITY;
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) take(v[u], base + u * kThreads, bv, bid);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bid, off);
+      take(ov, oi, bv, bid);
+    }
+    if (lane == 0) s_warp[warp] = Best{bv, bid};
+    __syncthreads();
+    if (warp == 0) {
+      Best m = lane < kThreads / 32 ? s_warp[lane] : Best{-INFINITY, INT_MAX};
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, m.v, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, m.id, off);
+        take(ov, oi, m.v, m.id);
+      }
+      if (lane == 0) s_slot[step & 1] = m;
+    }
+    cluster.sync();
+    // every CTA combines the partials of the whole cluster the same way
+    if (warp == 0) {
+      Best m{-INFINITY, INT_MAX};
+      if (lane < C) m = *cluster.map_shared_rank(&s_slot[step & 1], lane);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, m.v, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, m.id, off);
+        take(ov, oi, m.v, m.id);
+      }
+      if (lane == 0) {
+        int av = m.id;
+        if (av < 0 || av >= vocab) av = 0;  // only reachable with NaN rows
+        int match = INT_MAX;
+        if (L < max_depth) {
+          for (int k = 0; k < nk; ++k) {
+            const int c = s_kids[k];
+            if (s_tok[c] == av && c < match) match = c;
+          }
+        }
+        s_match = match;
+        s_arg = av;
+      }
+    }
+    __syncthreads();
+    a = s_arg;
+    const int match = s_match;
+    __syncthreads();  // everyone has read s_arg / s_match before they are reset
+    if (match == INT_MAX) break;
+    ++L;
+    cur = match;
+    if (tid == 0) s_path[L] = cur;
+  }
+  if (rank == 0 && tid == 0) {
+    accepted_len[b] = L;
+    bonus[b] = a;
+  }
+  if (rank == 0) {
+    int32_t* po = path + static_cast<long long>(b) * (max_depth + 1);
+    __syncthreads();
+    for (int i = tid; i <= max_depth; i += kThreads) po[i] = (i <= L) ? s_path[i] : -1;
+  }
+  // keep every CTA's shared memory alive until the last remote read of it has happened
+  cluster.sync();
+}
+
+}  // namespace acc
+
+cudaError_t launch_accept(const int32_t* token, const int32_t* parent, const float* logits, int batch,
+                          int num_nodes, int vocab, int max_depth, int32_t* accepted_len, int32_t* path,
+                          int32_t* bonus, int32_t* status, cudaStream_t stream) {
+  // cluster size: 16 CTAs when the device can co-schedule them, else the portable 8
+  static int cluster = 0;
+  if (cluster == 0) {
+    cluster = 8;
+    if (cudaFuncSetAttribute(acc::accept_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t probe = {};
+      probe.gridDim = dim3(acc::kMaxCluster);
+      probe.blockDim = dim3(acc::kThreads);
+      cudaLaunchAttribute at;
+      at.id = cudaLaunchAttributeClusterDimension;
+      at.val.clusterDim.x = acc::kMaxCluster;
+      at.val.clusterDim.y = 1;
+      at.val.clusterDim.z = 1;
+      probe.attrs = &at;
+      probe.numAttrs = 1;
+      int nclusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&nclusters, acc::accept_kernel, &probe) == cudaSuccess && nclusters > 0)
+        cluster = acc::kMaxCluster;
+    }
+    cudaGetLastError();  // clear a refused attribute / query
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(batch * cluster);
+  cfg.blockDim = dim3(acc::kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = cluster;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, acc::accept_kernel, token, parent, logits, num_nodes, vocab, max_depth,
+                            accepted_len, path, bonus, status);
+}
+
+}  // namespace jf

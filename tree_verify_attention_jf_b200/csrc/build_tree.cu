@@ -1,0 +1,508 @@
+// build_tree.cu -- best-first draft-tree construction under a token budget (sm_100a, SIMT).
+//
+// What it computes ("JetFlow: Breaking the Scaling Ceiling of Speculative Decoding with Parallel Tree
+// Drafting", technical summary section 2, tree construction): per-depth draft log-probabilities, then a
+// best-first expansion by cumulative log-probability until the tree holds `budget` nodes.
+//
+// Kernel 1 (row statistics, HBM-bound): one CTA per (row, 4096-entry chunk) of the [B, depths, V]
+// logits reads its chunk once (16-byte loads when the rows allow), and writes the chunk max, the
+// float64 sum of exp(x - chunk max) and the chunk's top-8 by (logit desc, id asc).
+// Kernel 2 (expansion, one CTA per sequence): merges the chunk partials into lse and the top-k per
+// depth (float64), then selects the budget's nodes.  Best-first popping by (key desc, depth asc,
+// parent index asc, rank asc) yields the budget-1 first nodes of that total order, so the kernel
+// computes them level-parallel instead of one pop at a time: because every depth-(d-1) node shares
+// the same top-k children (per-depth logits), the depth-d candidates are k copies of the sorted
+// depth-(d-1) list shifted by lp[d][r]; each candidate's rank among them follows from binary
+// searches, the best budget-1 of them are merged into the running global order, and the walk stops
+// once no deeper node can enter.  If its node pool would overflow (pathological ties), the CTA falls
+// back to popping one node at a time from per-(depth, rank) queues.
+#include <cfloat>
+
+#include "jf_device.cuh"
+#include "jf_internal.h"
+#include "jf_math.cuh"
+
+namespace jf {
+namespace build {
+
+constexpr int kThreads = 256;
+constexpr int kPerThread = kStatsChunk / kThreads;  // 16
+constexpr int kSlots = kMaxDepths * kMaxTopk / 32;  // queue slots per lane (16)
+
+struct Cand {
+  float v;
+  int id;
+};
+
+__device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
+  return a.v > b.v || (a.v == b.v && a.id < b.id);
+}
+
+__device__ __forceinline__ void cswap(Cand& a, Cand& b) {  // after: a better-or-equal than b
+  if (better(b, a)) {
+    const Cand t = a;
+    a = b;
+    b = t;
+  }
+}
+
+// keep t[] sorted best-first; insert x if it beats the last entry
+__device__ __forceinline__ void insert8(Cand (&t)[kMaxTopk], Cand x) {
+  if (!better(x, t[kMaxTopk - 1])) return;
+  t[kMaxTopk - 1] = x;
+#pragma unroll
+  for (int i = kMaxTopk - 1; i > 0; --i) cswap(t[i - 1], t[i]);
+}
+
+// t := best 8 of t U u (both sorted best-first), via a bitonic merge
+__device__ __forceinline__ void merge8(Cand (&t)[kMaxTopk], const Cand (&u)[kMaxTopk]) {
+#pragma unroll
+  for (int i = 0; i < kMaxTopk; ++i) {
+    const Cand o = u[kMaxTopk - 1 - i];
+    if (better(o, t[i])) t[i] = o;
+  }
+  // t is now bitonic; sort it best-first
+#pragma unroll
+  for (int span = kMaxTopk / 2; span > 0; span >>= 1) {
+#pragma unroll
+    for (int i = 0; i < kMaxTopk; ++i) {
+      if ((i & span) == 0) cswap(t[i], t[i + span]);
+    }
+  }
+}
+
+__device__ __forceinline__ void warp_merge8(Cand (&t)[kMaxTopk], int width) {
+  for (int off = width / 2; off > 0; off >>= 1) {
+    Cand u[kMaxTopk];
+#pragma unroll
+    for (int i = 0; i < kMaxTopk; ++i) {
+      u[i].v = __shfl_xor_sync(0xffffffffu, t[i].v, off);
+      u[i].id = __shfl_xor_sync(0xffffffffu, t[i].id, off);
+    }
+    merge8(t, u);
+  }
+}
+
+__device__ __forceinline__ double warp_sum_d(double x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+__device__ __forceinline__ float warp_max_f(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+  return x;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Kernel 1: chunk statistics.  grid = (chunks, batch * max_depth)
+// ------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads)
+    row_stats_kernel(const float* __restrict__ logits, int depths, int vocab, int max_depth,
+                     RowPartial* __restrict__ out) {
+  __shared__ float s_max[kThreads / 32];
+  __shared__ double s_sum[kThreads / 32];
+  __shared__ Cand s_top[kThreads / 32][kMaxTopk];
+  const int chunk = blockIdx.x, row = blockIdx.y;
+  const int b = row / max_depth, d = row - b * max_depth;
+  const float* x = logits + (static_cast<long long>(b) * depths + d) * vocab;
+  const int lo = chunk * kStatsChunk;
+  const int n = min(kStatsChunk, vocab - lo);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float v[kPerThread];
+  if (n == kStatsChunk && (reinterpret_cast<uintptr_t>(x + lo) & 15) == 0) {
+    // full, 16-byte aligned chunk: thread t reads float4 number t, t + 256, ...
+#pragma unroll
+    for (int j = 0; j < kPerThread / 4; ++j) {
+      const float4 q = __ldg(reinterpret_cast<const float4*>(x + lo) + j * kThreads + tid);
+      v[4 * j + 0] = q.x;
+      v[4 * j + 1] = q.y;
+      v[4 * j + 2] = q.z;
+      v[4 * j + 3] = q.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+      const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
+      v[j] = (i < n) ? __ldg(x + lo + i) : -INFINITY;
+    }
+  }
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) m = fmaxf(m, v[j]);
+  m = warp_max_f(m);
+  if (lane == 0) s_max[warp] = m;
+  __syncthreads();
+  m = s_max[0];
+#pragma unroll
+  for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, s_max[w]);
+  const double md = static_cast<double>(m);
+  double sum = 0.0;
+  Cand t[kMaxTopk];
+#pragma unroll
+  for (int i = 0; i < kMaxTopk; ++i) t[i] = Cand{-INFINITY, INT_MAX};
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
+    if (i < n) {
+      sum += exp_nonpos_f64(static_cast<double>(v[j]) - md);
+      insert8(t, Cand{v[j], lo + i});
+    }
+  }
+  sum = warp_sum_d(sum);
+  warp_merge8(t, 32);
+  if (lane == 0) {
+    s_sum[warp] = sum;
+#pragma unroll
+    for (int i = 0; i < kMaxTopk; ++i) s_top[warp][i] = t[i];
+  }
+  __syncthreads();
+  if (warp == 0) {
+    double ssum = (lane < kThreads / 32) ? s_sum[lane] : 0.0;
+    ssum = warp_sum_d(ssum);
+#pragma unroll
+    for (int i = 0; i < kMaxTopk; ++i) t[i] = (lane < kThreads / 32) ? s_top[lane][i] : Cand{-INFINITY, INT_MAX};
+    warp_merge8(t, 8);
+    if (lane == 0) {
+      RowPartial& o = out[static_cast<long long>(row) * gridDim.x + chunk];
+      o.sum = ssum;
+      o.m = m;
+      o.pad = 0;
+#pragma unroll
+      for (int i = 0; i < kMaxTopk; ++i) {
+        o.val[i] = t[i].v;
+        o.id[i] = t[i].id;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Kernel 2: merge + best-first expansion.  grid = batch, block = 256
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ unsigned long long ord_key(double k) {
+  const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(k));
+  return (bits >> 63) ? ~bits : (bits | 0x8000000000000000ull);
+}
+__device__ __forceinline__ double key_of_ord(unsigned long long o) {
+  const unsigned long long bits = (o >> 63) ? (o & 0x7fffffffffffffffull) : ~o;
+  return __longlong_as_double(static_cast<long long>(bits));
+}
+
+struct ExpandSmem {
+  double lp[kMaxDepths + 1][kMaxTopk];  // lp[d][r], d = 1..max_depth
+  int tok[kMaxDepths + 1][kMaxTopk];
+  double key[kMaxBudget];  // sequential fallback: node keys
+  int nsd[kMaxBudget];     // sequential fallback: next node of the same depth, in pop order
+  int tail[kMaxDepths + 1];
+  int n_kept, n_surv;
+};
+
+// Level-parallel selection state (dynamic shared memory).  Nodes are kept in a pool in creation
+// order; lists hold pool ids.
+constexpr int kPool = 4096;
+struct SelectSmem {
+  double pool_key[kPool];
+  int pool_par[kPool];  // parent's pool id, -1 = the root
+  int pool_dr[kPool];   // (depth << 8) | rank
+  int fidx[kPool];      // final node index of a pool entry
+  double prevkey[kMaxBudget];  // depth d-1 survivors, in order
+  int prevpid[kMaxBudget];
+  double lkey[kMaxBudget];     // best candidates of depth d, in order
+  int ljr[kMaxBudget];         // (parent position << 4) | rank
+  double gkey[2][kMaxBudget];  // global order so far (double-buffered)
+  int gpid[2][kMaxBudget];
+};
+
+size_t expand_dyn_smem() { return sizeof(SelectSmem); }
+
+// One warp pops the budget's nodes one at a time from per-(depth, rank) queues.  Queue (d, r) lists
+// the depth-(d-1) nodes in pop order paired with rank r; it is sorted by the pop order, so the best
+// candidate overall is the best queue head (found with redux.sync).
+__device__ void expand_sequential(ExpandSmem& s, int lane, int max_depth, int topk, int budget, int32_t* par_o,
+                                  int32_t* tok_o, float* sc_o, int32_t* dep_o) {
+  if (lane == 0) {
+    s.key[0] = 0.0;
+    s.nsd[0] = -1;
+    for (int i = 0; i <= kMaxDepths; ++i) s.tail[i] = -1;
+    s.tail[0] = 0;
+  }
+  __syncwarp();
+  const int nq = max_depth * topk;
+  const int nslots = (nq + 31) / 32;
+  unsigned long long qord[kSlots];
+  unsigned int qtie[kSlots];
+  int qnode[kSlots];
+#pragma unroll
+  for (int sl = 0; sl < kSlots; ++sl) {
+    const int q = sl * 32 + lane;
+    qord[sl] = 0ull;
+    qtie[sl] = 0xffffffffu;
+    qnode[sl] = -1;
+    if (sl < nslots && q < nq && q < topk) {
+      qnode[sl] = 0;
+      qord[sl] = ord_key(0.0 + s.lp[1][q]);
+      qtie[sl] = (1u << 13) | static_cast<unsigned>(q);
+    }
+  }
+  for (int n = 1; n < budget; ++n) {
+    unsigned long long best = 0ull;
+    unsigned int btie = 0xffffffffu;
+#pragma unroll
+    for (int sl = 0; sl < kSlots; ++sl) {
+      if (sl < nslots && (qord[sl] > best || (qord[sl] == best && qtie[sl] < btie))) {
+        best = qord[sl];
+        btie = qtie[sl];
+      }
+    }
+    const unsigned int hi = static_cast<unsigned int>(best >> 32);
+    const unsigned int mh = __reduce_max_sync(0xffffffffu, hi);
+    const unsigned int lo = (hi == mh) ? static_cast<unsigned int>(best) : 0u;
+    const unsigned int ml = __reduce_max_sync(0xffffffffu, lo);
+    const unsigned int tt = (hi == mh && static_cast<unsigned int>(best) == ml) ? btie : 0xffffffffu;
+    const unsigned int wt = __reduce_min_sync(0xffffffffu, tt);
+    if (mh == 0u && ml == 0u) break;
+    const int d = static_cast<int>(wt >> 13);
+    const int p = static_cast<int>((wt >> 3) & 1023u);
+    const int r = static_cast<int>(wt & 7u);
+    const double k = key_of_ord((static_cast<unsigned long long>(mh) << 32) | ml);
+    const int wq = (d - 1) * topk + r;
+    if (lane == 0) {
+      par_o[n] = p;
+      tok_o[n] = s.tok[d][r];
+      sc_o[n] = static_cast<float>(k);
+      if (dep_o) dep_o[n] = d;
+      s.key[n] = k;
+      s.nsd[n] = -1;
+      if (s.tail[d] >= 0) s.nsd[s.tail[d]] = n;
+      s.tail[d] = n;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int sl = 0; sl < kSlots; ++sl) {
+      if (sl < nslots && sl * 32 + lane == wq) {
+        const int nx = s.nsd[p];
+        qnode[sl] = nx;
+        if (nx >= 0) {
+          qord[sl] = ord_key(s.key[nx] + s.lp[d][r]);
+          qtie[sl] = (static_cast<unsigned>(d) << 13) | (static_cast<unsigned>(nx) << 3) | static_cast<unsigned>(r);
+        } else {
+          qord[sl] = 0ull;
+          qtie[sl] = 0xffffffffu;
+        }
+      }
+    }
+    if (d < max_depth) {
+#pragma unroll
+      for (int sl = 0; sl < kSlots; ++sl) {
+        const int q = sl * 32 + lane;
+        if (sl < nslots && q >= d * topk && q < (d + 1) * topk && qnode[sl] < 0) {
+          const int rr = q - d * topk;
+          qnode[sl] = n;
+          qord[sl] = ord_key(k + s.lp[d + 1][rr]);
+          qtie[sl] = (static_cast<unsigned>(d + 1) << 13) | (static_cast<unsigned>(n) << 3) | static_cast<unsigned>(rr);
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+    expand_kernel(const RowPartial* __restrict__ part, int nchunks, const int32_t* __restrict__ root_tokens,
+                  int max_depth, int topk, int budget, int32_t* __restrict__ parent, int32_t* __restrict__ token,
+                  float* __restrict__ score, int32_t* __restrict__ depth_out) {
+  __shared__ ExpandSmem s;
+  extern __shared__ __align__(16) uint8_t dyn[];
+  SelectSmem& q = *reinterpret_cast<SelectSmem*>(dyn);
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // ---- 1. per-depth lse (float64) and top-k
+  for (int d = 1 + warp; d <= max_depth; d += kThreads / 32) {
+    const RowPartial* rp = part + (static_cast<long long>(b) * max_depth + (d - 1)) * nchunks;
+    float m = -INFINITY;
+    for (int c = lane; c < nchunks; c += 32) m = fmaxf(m, rp[c].m);
+    m = warp_max_f(m);
+    const double md = static_cast<double>(m);
+    double sum = 0.0;
+    Cand t[kMaxTopk];
+#pragma unroll
+    for (int i = 0; i < kMaxTopk; ++i) t[i] = Cand{-INFINITY, INT_MAX};
+    for (int c = lane; c < nchunks; c += 32) {
+      sum += rp[c].sum * exp_nonpos_f64(static_cast<double>(rp[c].m) - md);
+      Cand u[kMaxTopk];
+#pragma unroll
+      for (int i = 0; i < kMaxTopk; ++i) u[i] = Cand{rp[c].val[i], rp[c].id[i]};
+      merge8(t, u);
+    }
+    sum = warp_sum_d(sum);
+    warp_merge8(t, 32);
+    if (lane == 0) {
+      const double lse = md + log(sum);
+#pragma unroll
+      for (int r = 0; r < kMaxTopk; ++r) {
+        s.lp[d][r] = static_cast<double>(t[r].v) - lse;
+        s.tok[d][r] = t[r].id;
+      }
+    }
+  }
+  int32_t* par_o = parent + static_cast<long long>(b) * budget;
+  int32_t* tok_o = token + static_cast<long long>(b) * budget;
+  float* sc_o = score + static_cast<long long>(b) * budget;
+  int32_t* dep_o = depth_out ? depth_out + static_cast<long long>(b) * budget : nullptr;
+  if (tid == 0) {
+    par_o[0] = -1;
+    tok_o[0] = root_tokens[b];
+    sc_o[0] = 0.f;
+    if (dep_o) dep_o[0] = 0;
+  }
+  const int T = budget - 1;
+  if (T == 0) return;
+  // ---- 2. level-parallel selection of the T best nodes in pop order
+  if (tid == 0) {
+    q.prevkey[0] = 0.0;
+    q.prevpid[0] = -1;
+  }
+  __syncthreads();
+  int n_prev = 1, g = 0, cur = 0, pool_base = 0;
+  bool overflow = false;
+  for (int d = 1; d <= max_depth; ++d) {
+    if (n_prev == 0) break;
+    const bool full = (g == T);
+    const double thr = full ? q.gkey[cur][T - 1] : 0.0;
+    if (full && !(q.prevkey[0] + s.lp[d][0] > thr)) break;  // no depth-d node can enter
+    if (tid == 0) {
+      s.n_kept = 0;
+      s.n_surv = 0;
+    }
+    __syncthreads();
+    const double* lpd = s.lp[d];
+    const int nc = n_prev * topk;
+    for (int idx = tid; idx < nc; idx += kThreads) {
+      const int j = idx / topk;
+      const int r = idx - j * topk;
+      const double kc = q.prevkey[j] + lpd[r];
+      if (full && !(kc > thr)) continue;  // cannot beat the current T-th node (ties go to shallower)
+      atomicAdd(&s.n_kept, 1);
+      int pos = j;  // candidates (j' < j, r) of its own list come first
+      for (int r2 = 0; r2 < topk; ++r2) {
+        if (r2 == r) continue;
+        int lo, hi;
+        if (r2 < r) { lo = j + 1; hi = n_prev; pos += 0; } else { lo = 0; hi = j; }
+        const double l2 = lpd[r2];
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          const double a = q.prevkey[mid] + l2;
+          const bool prec = a > kc || (a == kc && (mid < j || (mid == j && r2 < r)));
+          if (prec) lo = mid + 1; else hi = mid;
+        }
+        pos += lo;
+      }
+      if (pos < T) {
+        q.lkey[pos] = kc;
+        q.ljr[pos] = (j << 4) | r;
+      }
+    }
+    __syncthreads();
+    const int n_d = min(s.n_kept, T);
+    // merge the global order (g entries) with the depth-d list (n_d entries); equal keys: shallower first
+    for (int i = tid; i < g; i += kThreads) {
+      const double gk = q.gkey[cur][i];
+      int lo = 0, hi = n_d;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (q.lkey[mid] > gk) lo = mid + 1; else hi = mid;
+      }
+      const int pos = i + lo;
+      if (pos < T) {
+        q.gkey[cur ^ 1][pos] = gk;
+        q.gpid[cur ^ 1][pos] = q.gpid[cur][i];
+      }
+    }
+    for (int j = tid; j < n_d; j += kThreads) {
+      const double lk = q.lkey[j];
+      int lo = 0, hi = g;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (q.gkey[cur][mid] >= lk) lo = mid + 1; else hi = mid;
+      }
+      const int pos = j + lo;
+      if (pos < T) {
+        const int pid = pool_base + j;
+        atomicMax(&s.n_surv, j + 1);
+        if (pid < kPool) {
+          const int jr = q.ljr[j];
+          q.pool_key[pid] = lk;
+          q.pool_par[pid] = q.prevpid[jr >> 4];
+          q.pool_dr[pid] = (d << 8) | (jr & 15);
+        }
+        q.gkey[cur ^ 1][pos] = lk;
+        q.gpid[cur ^ 1][pos] = pid;
+      }
+    }
+    __syncthreads();
+    const int n_surv = s.n_surv;
+    if (pool_base + n_surv > kPool) {
+      overflow = true;
+      break;
+    }
+    for (int j = tid; j < n_surv; j += kThreads) {
+      q.prevkey[j] = q.lkey[j];
+      q.prevpid[j] = pool_base + j;
+    }
+    pool_base += n_surv;
+    n_prev = n_surv;
+    g = min(g + n_d, T);
+    cur ^= 1;
+    __syncthreads();
+  }
+  if (overflow || g < T) {
+    if (warp == 0) expand_sequential(s, lane, max_depth, topk, budget, par_o, tok_o, sc_o, dep_o);
+    return;
+  }
+  for (int i = tid; i < T; i += kThreads) q.fidx[q.gpid[cur][i]] = i + 1;
+  __syncthreads();
+  for (int i = tid; i < T; i += kThreads) {
+    const int pid = q.gpid[cur][i];
+    const int dr = q.pool_dr[pid];
+    const int d = dr >> 8, r = dr & 255;
+    const int pp = q.pool_par[pid];
+    par_o[i + 1] = pp < 0 ? 0 : q.fidx[pp];
+    tok_o[i + 1] = s.tok[d][r];
+    sc_o[i + 1] = static_cast<float>(q.pool_key[pid]);
+    if (dep_o) dep_o[i + 1] = d;
+  }
+}
+
+}  // namespace build
+
+size_t build_workspace_bytes(int batch, int depths, int vocab) {
+  (void)depths;
+  const long long nchunks = (static_cast<long long>(vocab) + kStatsChunk - 1) / kStatsChunk;
+  // sized for every depth row (max_depth <= depths)
+  return static_cast<size_t>(batch) * depths * nchunks * sizeof(RowPartial);
+}
+
+cudaError_t launch_build_tree(const float* logits, const int32_t* root_tokens, int batch, int depths, int vocab,
+                              int topk, int budget, int max_depth, int32_t* parent, int32_t* token, float* score,
+                              int32_t* depth, RowPartial* partials, int32_t* status, cudaStream_t stream) {
+  (void)status;
+  const int nchunks = (vocab + kStatsChunk - 1) / kStatsChunk;
+  dim3 g1(nchunks, batch * max_depth);
+  build::row_stats_kernel<<<g1, build::kThreads, 0, stream>>>(logits, depths, vocab, max_depth, partials);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  static bool attr_set = false;
+  const size_t dyn = build::expand_dyn_smem();
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(build::expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  build::expand_kernel<<<batch, build::kThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth, topk,
+                                                                budget, parent, token, score, depth);
+  return cudaGetLastError();
+}
+
+}  // namespace jf

@@ -1,0 +1,198 @@
+// jf_api.cu -- the C ABI of libjf.so (declared in include/jf.h): argument validation, TMA tensor-map
+// encoding, workspace carving and kernel launches.  Every check that needs no device data runs
+// before the first CUDA call, so a bad argument never launches anything.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/jf.h"
+#include "jf_internal.h"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int sm_count() {
+  static int counts[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// 3-D bf16 tensor map, dims innermost first, 128-byte swizzle, out-of-range boxes read as zero.
+bool encode_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
+               uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* jf_status_string(int status) {
+  switch (status) {
+    case JF_OK: return "JF_OK";
+    case JF_ERR_INVALID_ARG: return "JF_ERR_INVALID_ARG";
+    case JF_ERR_UNSUPPORTED: return "JF_ERR_UNSUPPORTED";
+    case JF_ERR_CUDA: return "JF_ERR_CUDA";
+    case JF_ERR_DEVICE_CHECK: return "JF_ERR_DEVICE_CHECK";
+    case JF_ERR_TIMEOUT: return "JF_ERR_TIMEOUT";
+    default: return "JF_ERR_UNKNOWN";
+  }
+}
+
+int jf_version(void) { return 10000; }
+
+size_t jf_tree_attention_workspace_size(int batch, int num_q_heads, int num_kv_heads, int total_nodes) {
+  (void)batch;
+  (void)num_q_heads;
+  (void)num_kv_heads;
+  (void)total_nodes;
+  return jf::AttnWorkspace::total;
+}
+
+jf_status jf_tree_attention(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                            int max_pages_per_seq, const int32_t* prefix_lens, const int32_t* tree_offsets,
+                            const int32_t* parent, int batch, int total_nodes, int num_q_heads, int num_kv_heads,
+                            int head_dim, int page_size, int num_pages, float sm_scale, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status, jf_stream_t stream) {
+  using namespace jf;
+  if (batch < 0 || total_nodes < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_pages_per_seq <= 0 ||
+      num_pages <= 0)
+    return JF_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return JF_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || page_size != kPageSize) return JF_ERR_UNSUPPORTED;
+  if (num_q_heads % num_kv_heads != 0) return JF_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8 && group != 16) return JF_ERR_UNSUPPORTED;
+  if (batch > kMaxAttnBatch) return JF_ERR_UNSUPPORTED;
+  if (static_cast<long long>(num_pages) * kPageSize >= (1ll << 31)) return JF_ERR_UNSUPPORTED;
+  if (batch == 0 || total_nodes == 0) return JF_OK;
+  if (!q || !k_cache || !v_cache || !block_table || !prefix_lens || !tree_offsets || !parent || !out || !workspace)
+    return JF_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(workspace, 256))
+    return JF_ERR_INVALID_ARG;
+  if (workspace_bytes < AttnWorkspace::total) return JF_ERR_INVALID_ARG;
+
+  const int sms = sm_count();
+  if (sms <= 0) return JF_ERR_CUDA;
+  const int grid = sms < kMaxGrid ? sms : kMaxGrid;
+
+  CUtensorMap tm_q, tm_k, tm_v;
+  const uint64_t row = kHeadDim * sizeof(__nv_bfloat16);  // 256 bytes
+  if (!encode_3d(&tm_q, q, kHeadDim, num_q_heads, total_nodes, row, row * num_q_heads, 64, group,
+                 kAttnRows / group))
+    return JF_ERR_CUDA;
+  const uint64_t slots = static_cast<uint64_t>(num_pages) * kPageSize;
+  if (!encode_3d(&tm_k, k_cache, kHeadDim, num_kv_heads, slots, row, row * num_kv_heads, 64, 1, kPageSize))
+    return JF_ERR_CUDA;
+  if (!encode_3d(&tm_v, v_cache, kHeadDim, num_kv_heads, slots, row, row * num_kv_heads, 64, 1, kPageSize))
+    return JF_ERR_CUDA;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  AttnParams p;
+  p.block_table = block_table;
+  p.prefix_lens = prefix_lens;
+  p.tree_offsets = tree_offsets;
+  p.parent = parent;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.counters = reinterpret_cast<int32_t*>(ws + AttnWorkspace::counters_off);
+  p.part_ok = reinterpret_cast<int32_t*>(ws + AttnWorkspace::ok_off);
+  p.part_ml = reinterpret_cast<float2*>(ws + AttnWorkspace::ml_off);
+  p.part_o = reinterpret_cast<float*>(ws + AttnWorkspace::o_off);
+  p.status = dev_status;
+  p.batch = batch;
+  p.total_nodes = total_nodes;
+  p.hq = num_q_heads;
+  p.hkv = num_kv_heads;
+  p.group = group;
+  p.max_pages = max_pages_per_seq;
+  p.num_pages = num_pages;
+  p.scale_log2 = sm_scale * 1.4426950408889634f;
+  if (launch_tree_attention(tm_q, tm_k, tm_v, p, grid, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JF_ERR_CUDA;
+  return JF_OK;
+}
+
+size_t jf_build_tree_workspace_size(int batch, int depths, int vocab, int topk) {
+  (void)topk;
+  if (batch <= 0 || depths <= 0 || vocab <= 0) return 0;
+  return jf::build_workspace_bytes(batch, depths, vocab);
+}
+
+jf_status jf_build_tree(const float* draft_logits, const int32_t* root_tokens, int batch, int depths, int vocab,
+                        int topk, int budget, int max_depth, int32_t* parent, int32_t* token, float* score,
+                        int32_t* depth, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                        jf_stream_t stream) {
+  using namespace jf;
+  if (batch < 0 || depths <= 0 || vocab <= 0 || topk <= 0 || budget <= 0 || max_depth <= 0)
+    return JF_ERR_INVALID_ARG;
+  if (topk > kMaxTopk || depths > kMaxDepths || budget > kMaxBudget) return JF_ERR_UNSUPPORTED;
+  if (topk > vocab || max_depth > depths) return JF_ERR_INVALID_ARG;
+  // the full topk-ary tree of depth max_depth must hold `budget` nodes
+  long long cap = 1, layer = 1;
+  for (int d = 1; d <= max_depth && cap < budget; ++d) {
+    layer = layer * topk;
+    if (layer > (1ll << 40)) layer = 1ll << 40;
+    cap += layer;
+  }
+  if (cap < budget) return JF_ERR_INVALID_ARG;
+  if (batch == 0) return JF_OK;
+  if (!draft_logits || !root_tokens || !parent || !token || !score || !workspace) return JF_ERR_INVALID_ARG;
+  if (!aligned(draft_logits, 4) || !aligned(workspace, 16)) return JF_ERR_INVALID_ARG;
+  if (workspace_bytes < build_workspace_bytes(batch, depths, vocab)) return JF_ERR_INVALID_ARG;
+  if (launch_build_tree(draft_logits, root_tokens, batch, depths, vocab, topk, budget, max_depth, parent, token,
+                        score, depth, static_cast<RowPartial*>(workspace), dev_status,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JF_ERR_CUDA;
+  return JF_OK;
+}
+
+jf_status jf_accept(const int32_t* token, const int32_t* parent, const float* target_logits, int batch,
+                    int num_nodes, int vocab, int max_depth, int32_t* accepted_len, int32_t* path,
+                    int32_t* bonus_token, int32_t* dev_status, jf_stream_t stream) {
+  using namespace jf;
+  if (batch < 0 || num_nodes <= 0 || vocab <= 0 || max_depth < 0) return JF_ERR_INVALID_ARG;
+  if (num_nodes > kMaxAcceptNodes || max_depth >= kMaxAcceptNodes) return JF_ERR_UNSUPPORTED;
+  if (batch == 0) return JF_OK;
+  if (!token || !parent || !target_logits || !accepted_len || !path || !bonus_token) return JF_ERR_INVALID_ARG;
+  if (!aligned(target_logits, 16)) return JF_ERR_INVALID_ARG;
+  if (launch_accept(token, parent, target_logits, batch, num_nodes, vocab, max_depth, accepted_len, path,
+                    bonus_token, dev_status, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JF_ERR_CUDA;
+  return JF_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// jf_internal.h -- declarations shared between the host entry points (jf_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace jf {
+
+constexpr int kHeadDim = 128;
+constexpr int kPageSize = 16;
+constexpr int kMaxTreeNodes = 256;          // nodes per sequence in jf_tree_attention
+constexpr int kAncWords = kMaxTreeNodes / 32;
+constexpr int kMaxAttnBatch = 2048;
+constexpr int kMaxGrid = 256;               // persistent CTAs (one per SM, capped)
+constexpr int kAttnRows = 128;              // rows of one M tile
+
+struct AttnParams {
+  const int32_t* block_table;
+  const int32_t* prefix_lens;
+  const int32_t* tree_offsets;
+  const int32_t* parent;
+  __nv_bfloat16* out;
+  float* lse;
+  float* part_o;    // [2*kMaxGrid][128][128] fp32 partial outputs
+  float2* part_ml;  // [2*kMaxGrid][128] (running max in log2 units, row sum)
+  int32_t* part_ok; // [2*kMaxGrid][128] 1 = the partial's sequence passed its device checks
+  int32_t* counters;  // [kMaxGrid][128] per-row arrival counters (zero between calls)
+  int32_t* status;
+  int batch, total_nodes, hq, hkv, group, max_pages, num_pages;
+  float scale_log2;
+};
+
+// Workspace layout of jf_tree_attention (offsets in bytes, each 256-aligned).
+struct AttnWorkspace {
+  static constexpr size_t counters_off = 0;
+  static constexpr size_t counters_bytes = sizeof(int32_t) * kMaxGrid * kAttnRows;
+  static constexpr size_t ok_off = counters_off + counters_bytes;
+  static constexpr size_t ok_bytes = sizeof(int32_t) * 2 * kMaxGrid * kAttnRows;
+  static constexpr size_t ml_off = ok_off + ok_bytes;
+  static constexpr size_t ml_bytes = sizeof(float2) * 2 * kMaxGrid * kAttnRows;
+  static constexpr size_t o_off = ml_off + ml_bytes;
+  static constexpr size_t o_bytes = sizeof(float) * 2 * kMaxGrid * kAttnRows * kHeadDim;
+  static constexpr size_t total = o_off + o_bytes;
+};
+
+size_t attention_smem_bytes();
+cudaError_t launch_tree_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                  const AttnParams& p, int grid, cudaStream_t stream);
+
+// ---- tree build
+constexpr int kMaxTopk = 8;
+constexpr int kMaxDepths = 64;
+constexpr int kMaxBudget = 1024;
+constexpr int kStatsChunk = 4096;  // vocab entries per row-statistics CTA
+
+struct RowPartial {  // one (row, chunk) of the draft logits
+  double sum;        // sum of exp(x - m) over the chunk, float64
+  float m;           // chunk max
+  int pad;
+  float val[kMaxTopk];
+  int id[kMaxTopk];
+};
+
+size_t build_workspace_bytes(int batch, int depths, int vocab);
+cudaError_t launch_build_tree(const float* logits, const int32_t* root_tokens, int batch, int depths, int vocab,
+                              int topk, int budget, int max_depth, int32_t* parent, int32_t* token, float* score,
+                              int32_t* depth, RowPartial* partials, int32_t* status, cudaStream_t stream);
+
+// ---- accept
+constexpr int kMaxAcceptNodes = 1024;
+cudaError_t launch_accept(const int32_t* token, const int32_t* parent, const float* logits, int batch,
+                          int num_nodes, int vocab, int max_depth, int32_t* accepted_len, int32_t* path,
+                          int32_t* bonus, int32_t* status, cudaStream_t stream);
+
+}  // namespace jf
