@@ -140,6 +140,30 @@ JF_API jf_status jf_build_tree(const float* draft_logits, const int32_t* root_to
                         size_t workspace_bytes, int32_t* dev_status, jf_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * jf_build_tree_noalloc -- jf_build_tree for callers that cannot allocate device memory.
+ *
+ * The pages describe no such call; it exists for hosts of this library that must not allocate at
+ * call time: for example a serving engine that hands all spare device memory to its KV-cache pool
+ * at start-up, or a plugin framework whose per-call hook is not allowed to allocate.  Such callers
+ * cannot provide jf_build_tree's workspace.  This variant takes no workspace: its scratch is a fixed
+ * 1 MiB array of device memory inside libjf.so, which every GPU that loads the library keeps until
+ * the process exits.
+ *
+ * Limit: batch * depths * ceil(vocab / 4096) * 80 bytes must fit in 1 MiB (for example batch 16 with
+ * 16 depths of a 151936-token vocabulary); larger calls return JF_ERR_UNSUPPORTED and launch nothing.
+ * The first call on each device looks up the array's device address with that device current
+ * (cudaGetSymbolAddress); make that first call before any stream capture.  Every call uses the same
+ * array and leaves its contents behind; nothing in it needs zeroing between calls, but two calls
+ * whose kernels overlap on the GPU (for example on two streams) corrupt each other's results, so
+ * such calls must be serialized.  All other arguments, outputs and errors are those of
+ * jf_build_tree.
+ * ------------------------------------------------------------------------------------------ */
+JF_API jf_status jf_build_tree_noalloc(const float* draft_logits, const int32_t* root_tokens, int batch,
+                                       int depths, int vocab, int topk, int budget, int max_depth,
+                                       int32_t* parent, int32_t* token, float* score, int32_t* depth,
+                                       int32_t* dev_status, jf_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * jf_accept -- greedy acceptance walk over the verified tree.
  *
  * Defines [JF section 1: the target verifies the drafted tokens in parallel and keeps the longest

@@ -17,7 +17,7 @@ def L():
 def test_exports_every_declared_symbol(L):
     names = _lib.declared_functions()
     assert set(names) == {"jf_status_string", "jf_version", "jf_tree_attention_workspace_size", "jf_tree_attention",
-                          "jf_build_tree_workspace_size", "jf_build_tree", "jf_accept"}
+                          "jf_build_tree_workspace_size", "jf_build_tree", "jf_build_tree_noalloc", "jf_accept"}
     for n in names:
         assert hasattr(L, n), n
 

@@ -17,6 +17,7 @@
 // once no deeper node can enter.  If its node pool would overflow (pathological ties), the CTA falls
 // back to popping one node at a time from per-(depth, rank) queues.
 #include <cfloat>
+#include <mutex>
 
 #include "jf_device.cuh"
 #include "jf_internal.h"
@@ -506,3 +507,47 @@ cudaError_t launch_build_tree(const float* logits, const int32_t* root_tokens, i
 }
 
 }  // namespace jf
+
+// ------------------------------------------------------------------------------------------------
+// jf_build_tree_noalloc: the row-statistics scratch of jf_build_tree in a fixed device array, for
+// callers that cannot allocate device memory when they call the library.
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB, held by every GPU that loads the library
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[64] = {};  // device address of g_noalloc_scratch, per device
+
+}  // namespace
+
+extern "C" JF_API jf_status jf_build_tree_noalloc(const float* draft_logits, const int32_t* root_tokens, int batch,
+                                                  int depths, int vocab, int topk, int budget, int max_depth,
+                                                  int32_t* parent, int32_t* token, float* score, int32_t* depth,
+                                                  int32_t* dev_status, jf_stream_t stream) {
+  if (batch < 0 || depths <= 0 || vocab <= 0) return JF_ERR_INVALID_ARG;
+  const unsigned long long chunks = (static_cast<unsigned long long>(vocab) + jf::kStatsChunk - 1) / jf::kStatsChunk;
+  const unsigned long long need =
+      static_cast<unsigned long long>(batch) * static_cast<unsigned long long>(depths) * chunks * sizeof(jf::RowPartial);
+  if (need > kNoAllocScratchBytes) return JF_ERR_UNSUPPORTED;
+  if (batch == 0)  // nothing to launch; let the common checks decide the status
+    return jf_build_tree(draft_logits, root_tokens, batch, depths, vocab, topk, budget, max_depth, parent, token,
+                         score, depth, nullptr, 0, dev_status, stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return JF_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      // In host code the array's name is only a stand-in; its device address comes from the runtime,
+      // looked up with this device current.
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return JF_ERR_CUDA;
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return jf_build_tree(draft_logits, root_tokens, batch, depths, vocab, topk, budget, max_depth, parent, token, score,
+                       depth, scratch, kNoAllocScratchBytes, dev_status, stream);
+}
