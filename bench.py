@@ -39,6 +39,7 @@ WORKLOADS = {
 HEAD_DIM = 128
 PAGE = 16
 L2_FLUSH_BYTES = 256 << 20
+LAUNCHES_PER_STEP = 5
 
 
 def peaks():
@@ -199,26 +200,54 @@ def run_gpu(args, cfg, rank, world, device):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
 
-    def step():
+    def build():
         api.build_tree(draft, roots, cfg["topk"], N, cfg["max_depth"], workspace=ws_build, out=tree)
-        ev[1].record(stream)
+
+    def attention():
         api.tree_attention(q, kc, vc, bt, prefix, offs, tree["parent"].view(-1), 1.0 / np.sqrt(HEAD_DIM), out=out,
                            workspace=ws_attn)
-        ev[2].record(stream)
+
+    def accept():
         api.accept(tree["token"], tree["parent"], tgt, cfg["max_depth"], out=acc_out)
 
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    def step():
+        build()
+        attention()
+        accept()
+
+    # eager warm-up (loads the library, sets kernel attributes), then one CUDA graph per timed region:
+    # the whole step, and each of its three calls alone for the per-kernel times
+    step()
+    torch.cuda.synchronize()
+    graphs = {}
+    for name, fn in (("step", step), ("build_tree", build), ("tree_attention", attention), ("accept", accept)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            fn()
+        graphs[name] = g
     for _ in range(args.warmup):
-        ev[0].record(stream)
-        step()
-        ev[3].record(stream)
+        graphs["step"].replay()
     torch.cuda.synchronize()
     expect_len = [len(p) - 1 for p in paths]
     got_len = acc_out["accepted_len"].cpu().tolist()
     if got_len != expect_len:
         raise RuntimeError(f"accepted lengths {got_len} != planted {expect_len}")
 
-    # ---- timed region: K steps, per-step events, L2 flushed between steps (outside the events)
+    # ---- timed region: K graph replays of the whole step, L2 flushed between steps (outside the events);
+    # then K replays of each call alone, for the per-kernel times
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def timed(g):
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            ev[0].record(stream)
+            g.replay()
+            ev[1].record(stream)
+            ev[1].synchronize()
+            ms.append(ev[0].elapsed_time(ev[1]))
+        return ms
+
     barrier(world)
     torch.cuda.synchronize()
     sampler = ClockSampler(torch.cuda.get_device_properties(device).uuid, os.path.join(ROOT, "gpurun_out",
@@ -226,20 +255,15 @@ def run_gpu(args, cfg, rank, world, device):
         if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(
             torch.cuda.get_device_properties(device).uuid, f"/tmp/jf_clocks_r{rank}.csv")
     time.sleep(0.3)
-    step_ms, attn_ms, build_ms, accept_ms = [], [], [], []
-    for _ in range(args.steps):
-        flush.zero_()
-        ev[0].record(stream)
-        step()
-        ev[3].record(stream)
-        ev[3].synchronize()
-        step_ms.append(ev[0].elapsed_time(ev[3]))
-        build_ms.append(ev[0].elapsed_time(ev[1]))
-        attn_ms.append(ev[1].elapsed_time(ev[2]))
-        accept_ms.append(ev[2].elapsed_time(ev[3]))
+    step_ms = timed(graphs["step"])
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop()
+    build_ms = timed(graphs["build_tree"])
+    attn_ms = timed(graphs["tree_attention"])
+    accept_ms = timed(graphs["accept"])
+    torch.cuda.synchronize()
+    del graphs
 
     # ---- e2e: the same step through the public API with host buffers; H2D of the step's inputs
     # (draft logits, tree queries, target logits) from pinned memory and D2H of its result inside
@@ -299,7 +323,8 @@ def main():
               "kv_heads": cfg["hkv"], "head_dim": HEAD_DIM, "prefix": cfg["prefix"], "page_size": PAGE,
               "budget": cfg["budget"], "topk": cfg["topk"], "max_depth": cfg["max_depth"], "vocab": cfg["vocab"],
               "step": "build_tree + tree_attention (one layer) + accept", "parallelism": f"replicas{world}",
-              "l2": "flushed between steps (256 MiB write outside the timed events)"}
+              "l2": "flushed between steps (256 MiB write outside the timed events)",
+              "launch": "one CUDA graph per step (host launch overhead outside the device timing)"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -362,7 +387,8 @@ def main():
         "time_share": shares,
         "e2e": {"value": nodes / (e2e_step * 1e-3), "unit": "nodes/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": 4 * args.steps,
+        # per step: row statistics + best-first expansion, attention + split combine, accept
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": r["clocks"],
         "cpu_baseline": cpu,
     }

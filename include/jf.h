@@ -90,12 +90,13 @@ JF_API int jf_version(void);
  *   out          bf16  [total_nodes, num_q_heads, head_dim]
  *   lse          fp32  [total_nodes, num_q_heads] or NULL
  * Supported: head_dim == 128, page_size == 16, num_q_heads % num_kv_heads == 0 with
- * Hq/Hkv in {1, 2, 4, 8, 16}, batch <= 2048.  q, k_cache, v_cache and out must be 16-byte aligned.
+ * Hq/Hkv in {1, 2, 4, 8, 16}, batch <= 1024.  q, k_cache, v_cache and out must be 16-byte aligned.
  * Cache slots beyond prefix_lens[b] + N_b in the last used page are never part of the result.
  *
  * workspace: at least jf_tree_attention_workspace_size(...) bytes of device memory, 256-byte
- * aligned, zero-filled before its FIRST use with this library; every call that completes leaves it
- * zeroed again where it needs zeros, so it can be reused across calls without a memset.
+ * aligned; it needs no initialisation and can be reused by consecutive calls on one stream.  A call
+ * launches the attention kernel and, right behind it on the same stream, a kernel that merges the
+ * partial results of work units the attention kernel split between CTAs.
  * ------------------------------------------------------------------------------------------ */
 JF_API size_t jf_tree_attention_workspace_size(int batch, int num_q_heads, int num_kv_heads, int total_nodes);
 

@@ -121,3 +121,36 @@ def test_pipeline_build_attend_accept():
     tgt, paths = synth.target_logits_with_path(79, tree["parent"], tree["token"], V)
     got = gpu_accept(tree["token"], tree["parent"], tgt, 16)
     assert got["accepted_len"].tolist() == [len(p) - 1 for p in paths]
+
+
+def test_build_and_accept_replay_in_a_cuda_graph():
+    """jf_build_tree (two launches) and jf_accept (a cluster launch) are capturable; a replay on fresh draft
+    logits written into the captured buffer gives the oracle's tree and accepted path."""
+    V, B = 8192, 3
+    x1, roots = synth.draft_logits(91, B, 16, V)
+    x2, _ = synth.draft_logits(92, B, 16, V)
+    xt = torch.from_numpy(np.ascontiguousarray(x1)).cuda()
+    rt = torch.from_numpy(np.ascontiguousarray(roots, dtype=np.int32)).cuda()
+    ws = api.build_tree_workspace(B, 16, V, 4, "cuda")
+    tree = api.build_tree(xt, rt, 4, 128, 16, workspace=ws)
+    torch.cuda.synchronize()
+    ref2 = oracle_build(x2, roots, 4, 128, 16)
+    tgt_np, paths = synth.target_logits_with_path(93, ref2["parent"], ref2["token"], V)
+    tgt = torch.from_numpy(tgt_np).cuda()
+    acc = dict(accepted_len=torch.empty(B, dtype=torch.int32, device="cuda"),
+               path=torch.empty(B, 17, dtype=torch.int32, device="cuda"),
+               bonus=torch.empty(B, dtype=torch.int32, device="cuda"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        api.build_tree(xt, rt, 4, 128, 16, workspace=ws, out=tree)
+        api.accept(tree["token"], tree["parent"], tgt, 16, out=acc)
+    xt.copy_(torch.from_numpy(np.ascontiguousarray(x2)))
+    g.replay()
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(tree["parent"].cpu().numpy(), ref2["parent"])
+    np.testing.assert_array_equal(tree["token"].cpu().numpy(), ref2["token"])
+    ref_len, ref_path, ref_bonus = oracle_accept(ref2["token"], ref2["parent"], tgt_np, 16)
+    np.testing.assert_array_equal(acc["accepted_len"].cpu().numpy(), ref_len)
+    np.testing.assert_array_equal(acc["path"].cpu().numpy(), ref_path)
+    np.testing.assert_array_equal(acc["bonus"].cpu().numpy(), ref_bonus)
+    assert acc["accepted_len"].cpu().tolist() == [len(p) - 1 for p in paths]

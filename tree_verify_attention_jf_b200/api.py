@@ -33,12 +33,12 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, device: torch.device) 
 
 
 class AttentionWorkspace:
-    """Zero-initialised scratch for :func:`tree_attention` (split-KV partials and per-row counters).
-    One per stream; reusable across calls (every completed call leaves it zeroed where needed)."""
+    """Scratch for :func:`tree_attention` (partial results of split work units).  One per stream;
+    needs no initialisation and is reusable across calls."""
 
     def __init__(self, device: torch.device):
         n = _lib.lib().jf_tree_attention_workspace_size(0, 0, 0, 0)
-        self.buf = torch.zeros(n, dtype=torch.uint8, device=device)
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device)
 
     @property
     def nbytes(self) -> int:

@@ -218,7 +218,10 @@ cudaError_t launch_accept(const int32_t* token, const int32_t* parent, const flo
                           int num_nodes, int vocab, int max_depth, int32_t* accepted_len, int32_t* path,
                           int32_t* bonus, int32_t* status, cudaStream_t stream) {
   // cluster size: 16 CTAs when the device can co-schedule them, else the portable 8
-  static int cluster = 0;
+  static std::atomic<int> cluster_of[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  int cluster = cluster_of[dev].load(std::memory_order_acquire);
   if (cluster == 0) {
     cluster = 8;
     if (cudaFuncSetAttribute(acc::accept_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
@@ -237,6 +240,7 @@ cudaError_t launch_accept(const int32_t* token, const int32_t* parent, const flo
         cluster = acc::kMaxCluster;
     }
     cudaGetLastError();  // clear a refused attribute / query
+    cluster_of[dev].store(cluster, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(batch * cluster);

@@ -48,41 +48,47 @@ __device__ __forceinline__ void cswap(Cand& a, Cand& b) {  // after: a better-or
 }
 
 // keep t[] sorted best-first; insert x if it beats the last entry
-__device__ __forceinline__ void insert8(Cand (&t)[kMaxTopk], Cand x) {
-  if (!better(x, t[kMaxTopk - 1])) return;
-  t[kMaxTopk - 1] = x;
+template <int K>
+__device__ __forceinline__ void insert_k(Cand (&t)[K], Cand x) {
+  if (!better(x, t[K - 1])) return;
+  t[K - 1] = x;
 #pragma unroll
-  for (int i = kMaxTopk - 1; i > 0; --i) cswap(t[i - 1], t[i]);
+  for (int i = K - 1; i > 0; --i) cswap(t[i - 1], t[i]);
 }
 
-// t := best 8 of t U u (both sorted best-first), via a bitonic merge
-__device__ __forceinline__ void merge8(Cand (&t)[kMaxTopk], const Cand (&u)[kMaxTopk]) {
+// t := best K of t U u (both sorted best-first), via a bitonic merge (K a power of two)
+template <int K>
+__device__ __forceinline__ void merge_k(Cand (&t)[K], const Cand (&u)[K]) {
 #pragma unroll
-  for (int i = 0; i < kMaxTopk; ++i) {
-    const Cand o = u[kMaxTopk - 1 - i];
+  for (int i = 0; i < K; ++i) {
+    const Cand o = u[K - 1 - i];
     if (better(o, t[i])) t[i] = o;
   }
   // t is now bitonic; sort it best-first
 #pragma unroll
-  for (int span = kMaxTopk / 2; span > 0; span >>= 1) {
+  for (int span = K / 2; span > 0; span >>= 1) {
 #pragma unroll
-    for (int i = 0; i < kMaxTopk; ++i) {
+    for (int i = 0; i < K; ++i) {
       if ((i & span) == 0) cswap(t[i], t[i + span]);
     }
   }
 }
 
-__device__ __forceinline__ void warp_merge8(Cand (&t)[kMaxTopk], int width) {
+template <int K>
+__device__ __forceinline__ void warp_merge_k(Cand (&t)[K], int width) {
   for (int off = width / 2; off > 0; off >>= 1) {
-    Cand u[kMaxTopk];
+    Cand u[K];
 #pragma unroll
-    for (int i = 0; i < kMaxTopk; ++i) {
+    for (int i = 0; i < K; ++i) {
       u[i].v = __shfl_xor_sync(0xffffffffu, t[i].v, off);
       u[i].id = __shfl_xor_sync(0xffffffffu, t[i].id, off);
     }
-    merge8(t, u);
+    merge_k<K>(t, u);
   }
 }
+
+__device__ __forceinline__ void merge8(Cand (&t)[kMaxTopk], const Cand (&u)[kMaxTopk]) { merge_k<kMaxTopk>(t, u); }
+__device__ __forceinline__ void warp_merge8(Cand (&t)[kMaxTopk], int width) { warp_merge_k<kMaxTopk>(t, width); }
 
 __device__ __forceinline__ double warp_sum_d(double x) {
 #pragma unroll
@@ -99,12 +105,15 @@ __device__ __forceinline__ float warp_max_f(float x) {
 // ------------------------------------------------------------------------------------------------
 // Kernel 1: chunk statistics.  grid = (chunks, batch * max_depth)
 // ------------------------------------------------------------------------------------------------
+// K: the per-chunk list length, the smallest power of two >= topk (only the best topk of a row can
+// ever become children, so shorter lists are exact and much cheaper to maintain).
+template <int K>
 __global__ void __launch_bounds__(kThreads)
     row_stats_kernel(const float* __restrict__ logits, int depths, int vocab, int max_depth,
                      RowPartial* __restrict__ out) {
   __shared__ float s_max[kThreads / 32];
   __shared__ double s_sum[kThreads / 32];
-  __shared__ Cand s_top[kThreads / 32][kMaxTopk];
+  __shared__ Cand s_top[kThreads / 32][K];
   const int chunk = blockIdx.x, row = blockIdx.y;
   const int b = row / max_depth, d = row - b * max_depth;
   const float* x = logits + (static_cast<long long>(b) * depths + d) * vocab;
@@ -140,31 +149,31 @@ __global__ void __launch_bounds__(kThreads)
   for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, s_max[w]);
   const double md = static_cast<double>(m);
   double sum = 0.0;
-  Cand t[kMaxTopk];
+  Cand t[K];
 #pragma unroll
-  for (int i = 0; i < kMaxTopk; ++i) t[i] = Cand{-INFINITY, INT_MAX};
+  for (int i = 0; i < K; ++i) t[i] = Cand{-INFINITY, INT_MAX};
 #pragma unroll
   for (int j = 0; j < kPerThread; ++j) {
     const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
     if (i < n) {
       sum += exp_nonpos_f64(static_cast<double>(v[j]) - md);
-      insert8(t, Cand{v[j], lo + i});
+      insert_k<K>(t, Cand{v[j], lo + i});
     }
   }
   sum = warp_sum_d(sum);
-  warp_merge8(t, 32);
+  warp_merge_k<K>(t, 32);
   if (lane == 0) {
     s_sum[warp] = sum;
 #pragma unroll
-    for (int i = 0; i < kMaxTopk; ++i) s_top[warp][i] = t[i];
+    for (int i = 0; i < K; ++i) s_top[warp][i] = t[i];
   }
   __syncthreads();
   if (warp == 0) {
     double ssum = (lane < kThreads / 32) ? s_sum[lane] : 0.0;
     ssum = warp_sum_d(ssum);
 #pragma unroll
-    for (int i = 0; i < kMaxTopk; ++i) t[i] = (lane < kThreads / 32) ? s_top[lane][i] : Cand{-INFINITY, INT_MAX};
-    warp_merge8(t, 8);
+    for (int i = 0; i < K; ++i) t[i] = (lane < kThreads / 32) ? s_top[lane][i] : Cand{-INFINITY, INT_MAX};
+    warp_merge_k<K>(t, 8);
     if (lane == 0) {
       RowPartial& o = out[static_cast<long long>(row) * gridDim.x + chunk];
       o.sum = ssum;
@@ -172,8 +181,8 @@ __global__ void __launch_bounds__(kThreads)
       o.pad = 0;
 #pragma unroll
       for (int i = 0; i < kMaxTopk; ++i) {
-        o.val[i] = t[i].v;
-        o.id[i] = t[i].id;
+        o.val[i] = i < K ? t[i < K ? i : 0].v : -INFINITY;
+        o.id[i] = i < K ? t[i < K ? i : 0].id : INT_MAX;
       }
     }
   }
@@ -491,15 +500,24 @@ cudaError_t launch_build_tree(const float* logits, const int32_t* root_tokens, i
   (void)status;
   const int nchunks = (vocab + kStatsChunk - 1) / kStatsChunk;
   dim3 g1(nchunks, batch * max_depth);
-  build::row_stats_kernel<<<g1, build::kThreads, 0, stream>>>(logits, depths, vocab, max_depth, partials);
+  if (topk <= 1)
+    build::row_stats_kernel<1><<<g1, build::kThreads, 0, stream>>>(logits, depths, vocab, max_depth, partials);
+  else if (topk <= 2)
+    build::row_stats_kernel<2><<<g1, build::kThreads, 0, stream>>>(logits, depths, vocab, max_depth, partials);
+  else if (topk <= 4)
+    build::row_stats_kernel<4><<<g1, build::kThreads, 0, stream>>>(logits, depths, vocab, max_depth, partials);
+  else
+    build::row_stats_kernel<8><<<g1, build::kThreads, 0, stream>>>(logits, depths, vocab, max_depth, partials);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  static bool attr_set = false;
+  static std::atomic<bool> attr_set[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
   const size_t dyn = build::expand_dyn_smem();
-  if (!attr_set) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(build::expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn));
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   build::expand_kernel<<<batch, build::kThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth, topk,
                                                                 budget, parent, token, score, depth);

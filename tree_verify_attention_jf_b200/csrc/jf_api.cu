@@ -28,15 +28,15 @@ EncodeTiledFn encode_fn() {
 }
 
 int sm_count() {
-  static int counts[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
-  if (counts[dev] == 0) {
-    int n = 0;
+  static std::atomic<int> counts[jf::kMaxDevices];
+  const int dev = jf::current_device();
+  if (dev < 0) return -1;
+  int n = counts[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-    counts[dev] = n;
+    counts[dev].store(n, std::memory_order_relaxed);
   }
-  return counts[dev];
+  return n;
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -128,7 +128,7 @@ jf_status jf_tree_attention(const void* q, const void* k_cache, const void* v_ca
   p.parent = parent;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  p.counters = reinterpret_cast<int32_t*>(ws + AttnWorkspace::counters_off);
+  p.units = reinterpret_cast<int4*>(ws + AttnWorkspace::units_off);
   p.part_ok = reinterpret_cast<int32_t*>(ws + AttnWorkspace::ok_off);
   p.part_ml = reinterpret_cast<float2*>(ws + AttnWorkspace::ml_off);
   p.part_o = reinterpret_cast<float*>(ws + AttnWorkspace::o_off);

@@ -7,15 +7,26 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace jf {
+
+// Kernel attributes (dynamic shared memory, cluster size) are per device: each launch function keeps one
+// flag per device and sets them the first time it launches on that device.
+constexpr int kMaxDevices = 64;
+inline int current_device() {
+  int d = -1;
+  return (cudaGetDevice(&d) == cudaSuccess && d >= 0 && d < kMaxDevices) ? d : -1;
+}
 
 constexpr int kHeadDim = 128;
 constexpr int kPageSize = 16;
 constexpr int kMaxTreeNodes = 256;          // nodes per sequence in jf_tree_attention
 constexpr int kAncWords = kMaxTreeNodes / 32;
-constexpr int kMaxAttnBatch = 2048;
+constexpr int kMaxAttnBatch = 1024;
 constexpr int kMaxGrid = 256;               // persistent CTAs (one per SM, capped)
 constexpr int kAttnRows = 128;              // rows of one M tile
+constexpr int kAttnQTiles = 2;              // M tiles per work unit (they share every K/V tile)
 
 struct AttnParams {
   const int32_t* block_table;
@@ -24,10 +35,10 @@ struct AttnParams {
   const int32_t* parent;
   __nv_bfloat16* out;
   float* lse;
-  float* part_o;    // [2*kMaxGrid][128][128] fp32 partial outputs
-  float2* part_ml;  // [2*kMaxGrid][128] (running max in log2 units, row sum)
-  int32_t* part_ok; // [2*kMaxGrid][128] 1 = the partial's sequence passed its device checks
-  int32_t* counters;  // [kMaxGrid][128] per-row arrival counters (zero between calls)
+  float* part_o;    // [2*kMaxGrid*2][32][128] float4 partial outputs (slot, column quad, row)
+  float2* part_ml;  // [2*kMaxGrid*2][128] (running max in log2 units, row sum)
+  int32_t* part_ok; // [2*kMaxGrid*2][128] 1 = the partial's sequence passed its device checks
+  int4* units;      // [kMaxGrid] descriptor of the split unit whose first CTA is i (c1, first node, nodes, kv head)
   int32_t* status;
   int batch, total_nodes, hq, hkv, group, max_pages, num_pages;
   float scale_log2;
@@ -35,14 +46,15 @@ struct AttnParams {
 
 // Workspace layout of jf_tree_attention (offsets in bytes, each 256-aligned).
 struct AttnWorkspace {
-  static constexpr size_t counters_off = 0;
-  static constexpr size_t counters_bytes = sizeof(int32_t) * kMaxGrid * kAttnRows;
-  static constexpr size_t ok_off = counters_off + counters_bytes;
-  static constexpr size_t ok_bytes = sizeof(int32_t) * 2 * kMaxGrid * kAttnRows;
+  static constexpr size_t kSlots = 2 * kMaxGrid * kAttnQTiles;  // (CTA, first/last segment, Q tile)
+  static constexpr size_t units_off = 0;
+  static constexpr size_t units_bytes = sizeof(int4) * kMaxGrid;
+  static constexpr size_t ok_off = units_off + ((units_bytes + 255) & ~size_t(255));
+  static constexpr size_t ok_bytes = sizeof(int32_t) * kSlots * kAttnRows;
   static constexpr size_t ml_off = ok_off + ok_bytes;
-  static constexpr size_t ml_bytes = sizeof(float2) * 2 * kMaxGrid * kAttnRows;
+  static constexpr size_t ml_bytes = sizeof(float2) * kSlots * kAttnRows;
   static constexpr size_t o_off = ml_off + ml_bytes;
-  static constexpr size_t o_bytes = sizeof(float) * 2 * kMaxGrid * kAttnRows * kHeadDim;
+  static constexpr size_t o_bytes = sizeof(float) * kSlots * kAttnRows * kHeadDim;
   static constexpr size_t total = o_off + o_bytes;
 };
 

@@ -6,17 +6,20 @@
 // its own root path (itself included), never to descendants or unrelated branches.
 //
 // How (B200-specific design, not taken from the pages, which only name an sm_90 paged kernel):
-//   * GQA packing: one M tile = 128 rows = (128 / g) tree nodes x g query heads of one kv head, so the
-//     K/V of that kv head is staged once for all its query heads.
-//   * Per CTA (persistent, one per SM): warp 0 loads Q with TMA (once per segment) and gathers K, warp 2
-//     gathers V: 128 keys (8 pages of 16 tokens) per tile, one TMA box per page and 64-column half,
-//     128-byte swizzled, gathered through the block table.  A box is only 2 KB, so the 16 boxes of a
-//     tile are issued by 16 lanes at once and K and V by separate warps.
-//     Warp 1 allocates tensor memory and issues tcgen05.mma: S = Q K^T (both operands from shared
-//     memory, K-major) into a double-buffered S in TMEM, and O += P V with P read straight from TMEM
-//     (aliasing S) and V as an MN-major shared-memory operand.  Warp 3 validates each segment and
-//     builds per-node 256-bit ancestor bitsets by pointer jumping.  Warps 4-7 (one thread per row) run
-//     the online softmax out of TMEM with a lazy rescale of O.
+//   * GQA packing: one M tile = 128 rows = (128 / g) tree nodes x g query heads of one kv head.  A work
+//     unit is a pair of M tiles of the same kv head: both are multiplied against every staged K/V tile,
+//     which halves the K/V traffic per unit of tensor-core work.
+//   * Per CTA (persistent, one per SM, 12 warps): warp 0 loads both Q tiles with TMA (once per
+//     segment) and gathers K, warp 2 gathers V: 128 keys (8 pages of 16 tokens) per tile, one TMA box
+//     per page and 64-column half, 128-byte swizzled, gathered through the block table; the 16 boxes of
+//     a tile are issued by 16 lanes at once.  Warp 1 allocates all 512 tensor-memory columns
+//     (S0 | S1 | O0 | O1) and issues tcgen05.mma: S_i = Q_i K^T (both operands from shared memory,
+//     K-major) and O_i += P_i V with P_i read straight from TMEM (aliasing S_i) and V as an MN-major
+//     shared-memory operand, in the order PV0(j), QK0(j+1), PV1(j), QK1(j+1) so that each softmax
+//     warpgroup works while the tensor core serves the other one.  Warp 3 validates each segment and
+//     builds per-node 256-bit ancestor bitsets by pointer jumping over warp shuffles.  Warps 4-7 and
+//     8-11 (one thread per row of M tile 0 / 1) run the online softmax out of TMEM with a lazy rescale
+//     of O, and the epilogue.
 //   * The tree mask only touches tiles that hold tree slots; prefix tiles are unmasked.
 //   * Work split: the flattened (unit, kv tile) space is cut into equal contiguous ranges, one per CTA
 //     (stream-K).  A unit cut between CTAs writes fp32 partials; per row, the last CTA to finish (an
@@ -32,42 +35,45 @@ constexpr int kBM = 128;             // rows per M tile
 constexpr int kBN = 128;             // keys per KV tile
 constexpr int kPagesPerTile = kBN / kPage;
 constexpr int kStages = 2;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kHalfBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kTileBytes = 2 * kHalfBytes;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmO = 256;  // S buffers at columns 0 and 128, O at 256
+constexpr uint32_t kTmS = 0;    // S_i at column 128 * i
+constexpr uint32_t kTmO = 256;  // O_i at column 256 + 128 * i
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow up to 2^8 before O is rescaled
 
 struct __align__(1024) Smem {
-  uint8_t q[kTileBytes];
+  uint8_t q[kAttnQTiles][kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
   uint32_t anc[2][kMaxTreeNodes][kAncWords];
-  uint32_t anc_tmp[kMaxTreeNodes][kAncWords];
-  int32_t jmp[2][kMaxTreeNodes];
   long long cum_work[kMaxAttnBatch + 1];
   long long scan_warp[kThreads / 32];
   uint64_t bar_qfull, bar_qempty;
   uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
-  uint64_t bar_sfull[2], bar_pfull[2], bar_pvdone[2];  // pvdone[j & 1] completes when PV(j) is done
+  uint64_t bar_sfull[kAttnQTiles], bar_pfull[kAttnQTiles], bar_pvdone[kAttnQTiles];
   uint64_t bar_metafull[2], bar_metaempty[2];
   uint32_t tmem_base;
   int meta_valid[2];
-  int meta_tree[2];
   int meta_ctl;
   int abort_flag;
   int bad_meta;
 };
 
 struct Seg {
-  int b, kvh, mt, kb, ke;  // kv tiles [kb, ke) of unit (b, kvh, mt)
+  int b, kvh, mp, kb, ke;  // kv tiles [kb, ke) of unit (b, kvh, M-tile pair mp)
   int P, N, off, kt;       // prefix length, nodes, first global node, kv tiles of the sequence
-  int c0, c1, slot;        // CTAs sharing the unit; this CTA's partial slot
+  int c0, c1, slot;        // CTAs sharing the unit; this CTA's partial slot (times kAttnQTiles)
 };
 
 __device__ __forceinline__ int cta_of(long long x, long long W, int G) {
   return static_cast<int>(((x + 1) * G - 1) / W);
+}
+
+__device__ __forceinline__ int pairs_of(int N, int group) {
+  const int mtn = (N * group + kBM - 1) / kBM;
+  return (mtn + kAttnQTiles - 1) / kAttnQTiles;
 }
 
 struct SegIter {
@@ -81,12 +87,12 @@ struct SegIter {
     g.off = p.tree_offsets[b];
     g.N = p.tree_offsets[b + 1] - g.off;
     g.kt = (g.P + g.N + kBN - 1) / kBN;
-    const int mtn = (g.N * p.group + kBM - 1) / kBM;
+    const int mpn = pairs_of(g.N, p.group);
     const long long local = x - s.cum_work[b];
     const long long unit = local / g.kt;
     g.kb = static_cast<int>(local - unit * g.kt);
-    g.kvh = static_cast<int>(unit / mtn);
-    g.mt = static_cast<int>(unit - static_cast<long long>(g.kvh) * mtn);
+    g.kvh = static_cast<int>(unit / mpn);
+    g.mp = static_cast<int>(unit - static_cast<long long>(g.kvh) * mpn);
     const long long u0 = s.cum_work[b] + unit * g.kt, u1 = u0 + g.kt;
     const long long e = xend < u1 ? xend : u1;
     g.ke = g.kb + static_cast<int>(e - x);
@@ -97,6 +103,8 @@ struct SegIter {
     return true;
   }
 };
+
+__device__ __forceinline__ int slot_of(int c, int c0) { return (c == c0) ? 2 * c + 1 : 2 * c; }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const bool ok = mbar_wait(bar, parity, abort);
@@ -109,7 +117,7 @@ __device__ __forceinline__ void set_abort(Smem& s, const AttnParams& p) {
 }
 
 // ------------------------------------------------------------------------------------------------
-// Plan: per-sequence work (kv heads x M tiles x kv tiles), exclusive prefix sum in shared memory,
+// Plan: per-sequence work (kv heads x M-tile pairs x kv tiles), exclusive prefix sum in shared memory,
 // validation of the batch-level metadata.  Every CTA computes the same plan.
 // ------------------------------------------------------------------------------------------------
 __device__ void build_plan(Smem& s, const AttnParams& p) {
@@ -131,11 +139,9 @@ __device__ void build_plan(Smem& s, const AttnParams& p) {
     }
     if (N == 0) continue;
     const long long kt = (static_cast<long long>(P) + N + kBN - 1) / kBN;
-    const long long mtn = (static_cast<long long>(N) * p.group + kBM - 1) / kBM;
-    local += static_cast<long long>(p.hkv) * mtn * kt;
+    local += static_cast<long long>(p.hkv) * pairs_of(N, p.group) * kt;
   }
   if (bad) atomicOr(&s.bad_meta, 1);
-  // block-wide exclusive scan of `local`
   long long incl = local;
   for (int o = 1; o < 32; o <<= 1) {
     const long long v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -152,15 +158,14 @@ __device__ void build_plan(Smem& s, const AttnParams& p) {
     const int N = p.tree_offsets[b + 1] - p.tree_offsets[b];
     if (P < 0 || N <= 0 || N > kMaxTreeNodes) continue;
     const long long kt = (static_cast<long long>(P) + N + kBN - 1) / kBN;
-    const long long mtn = (static_cast<long long>(N) * p.group + kBM - 1) / kBM;
-    run += static_cast<long long>(p.hkv) * mtn * kt;
+    run += static_cast<long long>(p.hkv) * pairs_of(N, p.group) * kt;
   }
   if (tid == kThreads - 1) s.cum_work[B] = run;
   __syncthreads();
 }
 
 // ------------------------------------------------------------------------------------------------
-// Warps 0 and 2: K / V gathers (warp 0 also loads Q)
+// Warps 0 and 2: K / V gathers (warp 0 also loads the Q tiles)
 // ------------------------------------------------------------------------------------------------
 __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_v, const CUtensorMap* tm_q,
                             const CUtensorMap* tm_kv) {
@@ -174,11 +179,12 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
   while (iter.next(s, p, g)) {
     if (!is_v) {
       if (!warp_wait(&s.bar_qempty, (sidx & 1) ^ 1, abort)) return set_abort(s, p);
-      if (lane == 0) {
-        const int node0 = g.off + g.mt * nodes_per_tile;
-        mbar_arrive_expect_tx(&s.bar_qfull, kTileBytes);
-        tma_load_3d(s.q, tm_q, &s.bar_qfull, 0, g.kvh * p.group, node0);
-        tma_load_3d(s.q + kHalfBytes, tm_q, &s.bar_qfull, 64, g.kvh * p.group, node0);
+      if (lane == 0) mbar_arrive_expect_tx(&s.bar_qfull, kAttnQTiles * kTileBytes);
+      __syncwarp();
+      if (lane < 2 * kAttnQTiles) {  // lane: Q tile lane / 2, half lane % 2
+        const int qt = lane >> 1, half = lane & 1;
+        const int node0 = g.off + (g.mp * kAttnQTiles + qt) * nodes_per_tile;
+        tma_load_3d(s.q[qt] + half * kHalfBytes, tm_q, &s.bar_qfull, half * 64, g.kvh * p.group, node0);
       }
     }
     const int npg = (g.P + g.N + kPage - 1) / kPage;
@@ -228,46 +234,26 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
 // ------------------------------------------------------------------------------------------------
 // Warp 1: tcgen05.mma issuer
 // ------------------------------------------------------------------------------------------------
-struct PendingPV {
-  uint32_t it;
-  int st, first, zero_from;
-};
-
-__device__ __forceinline__ bool issue_pv(Smem& s, const AttnParams& p, uint32_t tmem, const PendingPV& pv) {
-  const int lane = threadIdx.x & 31;
-  volatile int* abort = &s.abort_flag;
-  const int sb = pv.it & 1;
-  if (!warp_wait(&s.bar_pfull[sb], (pv.it >> 1) & 1, abort)) return false;
-  if (!warp_wait(&s.bar_vfull[pv.st], (pv.it / kStages) & 1, abort)) return false;
-  if (pv.zero_from < kBN) {
-    // Keys beyond the sequence's last slot: clear their V rows so stale cache contents (even NaN)
-    // cannot reach the output through 0 * V.  A whole 128-byte row is cleared, so the swizzle does
-    // not matter.
-    uint8_t* vb = s.v[pv.st];
-    const int nchunks = (kBN - pv.zero_from) * 16;
-    for (int i = lane; i < nchunks; i += 32) {
-      const int row = pv.zero_from + (i >> 4);
-      const int half = (i >> 3) & 1;
-      const int c = i & 7;
-      *reinterpret_cast<uint4*>(vb + half * kHalfBytes + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
-  }
-  __syncwarp();
-  tc_fence_after();
-  if (lane == 0) {
-    constexpr uint32_t idesc = idesc_bf16_f32(kBM, 128, false, true);
-    const uint32_t vaddr = smem_u32(s.v[pv.st]);
+__device__ __forceinline__ void issue_qk(const Smem& s, uint32_t tmem, int qt, int st) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, false, false);
+  const uint32_t qaddr = smem_u32(s.q[qt]);
+  const uint32_t kaddr = smem_u32(s.k[st]);
 #pragma unroll
-    for (int kk = 0; kk < kBN / 16; ++kk) {
-      const uint64_t bdesc = smem_desc_sw128(vaddr + kk * 2048, kHalfBytes, 1024);
-      mma_ts(tmem + kTmO, tmem + sb * 128 + kk * 8, bdesc, idesc, (pv.first && kk == 0) ? 0u : 1u);
-    }
-    mma_commit(&s.bar_pvdone[pv.it & 1]);
-    mma_commit(&s.bar_vempty[pv.st]);
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+    mma_ss(tmem + kTmS + qt * 128, smem_desc_sw128(qaddr + off, 16, 1024), smem_desc_sw128(kaddr + off, 16, 1024),
+           idesc, kk > 0 ? 1u : 0u);
   }
-  __syncwarp();
-  return true;
+}
+
+__device__ __forceinline__ void issue_pv(const Smem& s, uint32_t tmem, int qt, int st, bool first) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kBM, 128, false, true);
+  const uint32_t vaddr = smem_u32(s.v[st]);
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk) {
+    mma_ts(tmem + kTmO + qt * 128, tmem + kTmS + qt * 128 + kk * 8, smem_desc_sw128(vaddr + kk * 2048, kHalfBytes, 1024),
+           idesc, (first && kk == 0) ? 0u : 1u);
+  }
 }
 
 __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t tmem) {
@@ -275,126 +261,146 @@ __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t 
   volatile int* abort = &s.abort_flag;
   Seg g;
   uint32_t it = 0, sidx = 0;
-  bool have_prev = false;
-  PendingPV prev{};
-  constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
-  const uint32_t qaddr = smem_u32(s.q);
   while (iter.next(s, p, g)) {
     if (!warp_wait(&s.bar_qfull, sidx & 1, abort)) return set_abort(s, p);
     for (int t = g.kb; t < g.ke; ++t, ++it) {
       const int st = it % kStages;
-      const int sb = it & 1;
-      if (!warp_wait(&s.bar_kfull[st], (it / kStages) & 1, abort)) return set_abort(s, p);
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t kaddr = smem_u32(s.k[st]);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          const uint64_t adesc = smem_desc_sw128(qaddr + off, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(kaddr + off, 16, 1024);
-          mma_ss(tmem + sb * 128, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+      if (t == g.kb) {  // S of the segment's first tile for both Q tiles
+        if (!warp_wait(&s.bar_kfull[st], (it / kStages) & 1, abort)) return set_abort(s, p);
+        tc_fence_after();
+        if (lane == 0) {
+          issue_qk(s, tmem, 0, st);
+          mma_commit(&s.bar_sfull[0]);
+          issue_qk(s, tmem, 1, st);
+          mma_commit(&s.bar_sfull[1]);
+          mma_commit(&s.bar_kempty[st]);
+          if (t == g.ke - 1) mma_commit(&s.bar_qempty);
         }
-        mma_commit(&s.bar_sfull[sb]);
-        mma_commit(&s.bar_kempty[st]);
-        if (t == g.ke - 1) mma_commit(&s.bar_qempty);
+        __syncwarp();
       }
-      __syncwarp();
-      if (have_prev && !issue_pv(s, p, tmem, prev)) return set_abort(s, p);
+      const bool has_next = t + 1 < g.ke;
+      const int st1 = (it + 1) % kStages;
+      if (has_next && !warp_wait(&s.bar_kfull[st1], ((it + 1) / kStages) & 1, abort)) return set_abort(s, p);
+      if (!warp_wait(&s.bar_vfull[st], (it / kStages) & 1, abort)) return set_abort(s, p);
       const int zf = g.P + g.N - t * kBN;  // first row of this tile past the sequence
-      prev.it = it;
-      prev.st = st;
-      prev.first = (t == g.kb);
-      prev.zero_from = zf < 0 ? 0 : zf;
-      have_prev = true;
+      if (zf < kBN) {
+        // Keys beyond the sequence's last slot: clear their V rows so stale cache contents (even NaN)
+        // cannot reach the output through 0 * V.  A whole 128-byte row is cleared, so the swizzle does
+        // not matter.
+        uint8_t* vb = s.v[st];
+        const int z0 = zf < 0 ? 0 : zf;
+        const int nchunks = (kBN - z0) * 16;
+        for (int i = lane; i < nchunks; i += 32) {
+          const int row = z0 + (i >> 4);
+          const int half = (i >> 3) & 1;
+          const int c = i & 7;
+          *reinterpret_cast<uint4*>(vb + half * kHalfBytes + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      for (int qt = 0; qt < kAttnQTiles; ++qt) {
+        if (!warp_wait(&s.bar_pfull[qt], it & 1, abort)) return set_abort(s, p);
+        tc_fence_after();
+        if (lane == 0) {
+          issue_pv(s, tmem, qt, st, t == g.kb);
+          mma_commit(&s.bar_pvdone[qt]);
+          if (qt == kAttnQTiles - 1) mma_commit(&s.bar_vempty[st]);
+          if (has_next) {
+            issue_qk(s, tmem, qt, st1);
+            mma_commit(&s.bar_sfull[qt]);
+            if (qt == kAttnQTiles - 1) {
+              mma_commit(&s.bar_kempty[st1]);
+              if (t + 1 == g.ke - 1) mma_commit(&s.bar_qempty);
+            }
+          }
+        }
+        __syncwarp();
+      }
     }
     ++sidx;
   }
-  if (have_prev && !issue_pv(s, p, tmem, prev)) return set_abort(s, p);
 }
 
 // ------------------------------------------------------------------------------------------------
-// Warp 3: per-segment validation and ancestor bitsets (pointer jumping over parent[])
+// Warp 3: per-segment validation and ancestor bitsets
 // ------------------------------------------------------------------------------------------------
 __device__ void metadata(Smem& s, const AttnParams& p, SegIter iter) {
-  const int mt = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   volatile int* abort = &s.abort_flag;
   Seg g;
   uint32_t sidx = 0;
   while (iter.next(s, p, g)) {
     const int buf = sidx & 1;
-    if (mt == 0) {
+    if (lane == 0) {
       const bool ok = mbar_wait(&s.bar_metaempty[buf], ((sidx >> 1) & 1) ^ 1, abort);
       s.meta_ctl = ok ? 1 : 0;
       if (!ok) set_abort(s, p);
     }
     __syncwarp();
     if (s.meta_ctl == 0) return;
-    // --- validation
+    // --- validation: parent indices, capacity, the page ids this segment reads
     int bad = 0;
     const int npg = (g.P + g.N + kPage - 1) / kPage;
     if (static_cast<long long>(g.P) + g.N > static_cast<long long>(p.max_pages) * kPage) bad = 1;
     const int32_t* par = p.parent + g.off;
-    for (int i = mt; i < g.N; i += 32) {
+    for (int i = lane; i < g.N; i += 32) {
       const int pi = par[i];
       if (pi < -1 || pi >= i) bad = 1;
     }
     const int32_t* bt = p.block_table + static_cast<long long>(g.b) * p.max_pages;
-    const int pg0 = g.kb * kPagesPerTile;
     int pg1 = g.ke * kPagesPerTile;
     if (pg1 > npg) pg1 = npg;
     if (pg1 > p.max_pages) pg1 = p.max_pages;
-    for (int pg = pg0 + mt; pg < pg1; pg += 32) {
+    for (int pg = g.kb * kPagesPerTile + lane; pg < pg1; pg += 32) {
       const int v = bt[pg];
       if (v < 0 || v >= p.num_pages) bad = 1;
     }
-    if (mt == 0) s.meta_valid[buf] = 1;
-    __syncwarp();
-    if (bad) {
-      s.meta_valid[buf] = 0;
-      report(p.status, JF_ERR_DEVICE_CHECK);
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      s.meta_valid[buf] = bad ? 0 : 1;
+      if (bad) report(p.status, JF_ERR_DEVICE_CHECK);
     }
-    // --- ancestor bitsets, only if the segment reaches the tree slots
-    const bool tree = static_cast<long long>(g.ke) * kBN > g.P;
-    if (tree) {
-      uint32_t(*A)[kAncWords] = s.anc[buf];
-      for (int i = mt; i < g.N; i += 32) {
-        const int pi = par[i];
-        s.jmp[0][i] = (pi >= 0 && pi < i) ? pi : -1;
+    // --- ancestor bitsets (only needed when the segment reaches the tree slots).  Nodes are taken
+    // 32 at a time in index order; a node whose parent lies in an earlier chunk starts from the
+    // parent's finished bitset, the others resolve their in-chunk chain by pointer jumping over warp
+    // shuffles (5 rounds cover 32 levels).
+    if (static_cast<long long>(g.ke) * kBN > g.P) {
+      for (int base = 0; base < g.N; base += 32) {
+        const int i = base + lane;
+        uint32_t a[kAncWords];
 #pragma unroll
-        for (int w = 0; w < kAncWords; ++w) A[i][w] = (w == (i >> 5)) ? (1u << (i & 31)) : 0u;
-      }
-      __syncwarp();
-      // After round r every node holds its ancestors at distance < 2^r; 8 rounds cover 256 levels.
-      uint32_t(*src)[kAncWords] = s.anc[buf];
-      uint32_t(*dst)[kAncWords] = s.anc_tmp;
-      int cur = 0;
-      for (int round = 0; round < 8; ++round) {
-        for (int i = mt; i < g.N; i += 32) {
-          const int j = s.jmp[cur][i];
-          uint4 a0 = *reinterpret_cast<const uint4*>(&src[i][0]);
-          uint4 a1 = *reinterpret_cast<const uint4*>(&src[i][4]);
-          int jj = -1;
-          if (j >= 0) {
-            const uint4 b0 = *reinterpret_cast<const uint4*>(&src[j][0]);
-            const uint4 b1 = *reinterpret_cast<const uint4*>(&src[j][4]);
-            a0.x |= b0.x; a0.y |= b0.y; a0.z |= b0.z; a0.w |= b0.w;
-            a1.x |= b1.x; a1.y |= b1.y; a1.z |= b1.z; a1.w |= b1.w;
-            jj = s.jmp[cur][j];
+        for (int w = 0; w < kAncWords; ++w) a[w] = 0u;
+        int jl = -1;  // lane of the next in-chunk ancestor still to merge
+        if (i < g.N) {
+          a[i >> 5] = 1u << (i & 31);
+          int pi = par[i];
+          if (pi >= i) pi = -1;  // invalid parents were flagged above; keep the walk in range
+          if (pi >= 0 && pi < base) {
+#pragma unroll
+            for (int w = 0; w < kAncWords; ++w) a[w] |= s.anc[buf][pi][w];
+          } else if (pi >= base) {
+            jl = pi - base;
           }
-          *reinterpret_cast<uint4*>(&dst[i][0]) = a0;
-          *reinterpret_cast<uint4*>(&dst[i][4]) = a1;
-          s.jmp[cur ^ 1][i] = jj;
+        }
+#pragma unroll
+        for (int round = 0; round < 5; ++round) {
+          const int src = jl >= 0 ? jl : lane;
+#pragma unroll
+          for (int w = 0; w < kAncWords; ++w) {
+            const uint32_t o = __shfl_sync(0xffffffffu, a[w], src);
+            if (jl >= 0) a[w] |= o;
+          }
+          const int oj = __shfl_sync(0xffffffffu, jl, src);
+          jl = jl >= 0 ? oj : -1;
+        }
+        if (i < g.N) {
+#pragma unroll
+          for (int w = 0; w < kAncWords; ++w) s.anc[buf][i][w] = a[w];
         }
         __syncwarp();
-        uint32_t(*t)[kAncWords] = src;
-        src = dst;
-        dst = t;
-        cur ^= 1;
       }
-      // 8 rounds (even): the result is back in s.anc[buf]
     }
-    if (mt == 0) s.meta_tree[buf] = tree ? 1 : 0;
     __threadfence_block();
     mbar_arrive(&s.bar_metafull[buf]);
     ++sidx;
@@ -402,7 +408,7 @@ __device__ void metadata(Smem& s, const AttnParams& p, SegIter iter) {
 }
 
 // ------------------------------------------------------------------------------------------------
-// Warps 4-7: online softmax (one thread per row) and the epilogue
+// Warps 4-11: online softmax (one thread per row of M tile 0 or 1) and the epilogue
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const float* o, float inv_l) {
 #pragma unroll
@@ -445,15 +451,55 @@ __device__ __forceinline__ uint32_t vis_word(int slot0, int P, int N, bool row_v
 }
 
 // Partial outputs are stored column-quad-major so that a warp's 32 rows touch 512 contiguous bytes:
-// float4 index ((slot * 32 + c4) * 128 + row).
+// float4 index ((slot * 32 + c4) * 128 + row), slot = 2 * (segment slot) + Q tile.
 __device__ __forceinline__ float4* part_ptr(const AttnParams& p, int slot, int c4, int r) {
   return reinterpret_cast<float4*>(p.part_o) + (static_cast<long long>(slot) * 32 + c4) * kBM + r;
 }
 
-__device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uint32_t tmem) {
-  const int r = threadIdx.x - 128;  // row of the M tile == TMEM lane
+__device__ __forceinline__ float slice_max(const uint32_t (&sr)[32], uint32_t vis) {
+  float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+  if (vis == 0xffffffffu) {
+#pragma unroll
+    for (int c = 0; c < 32; c += 8) {
+      a0 = fmax3(a0, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
+      a1 = fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+      a2 = fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+      a3 = fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+      if ((vis >> c) & 1u) a0 = fmaxf(a0, __uint_as_float(sr[c]));
+  }
+  return fmax3(a0, a1, fmaxf(a2, a3));
+}
+
+// P = 2^(s * scale - m) for one 32-column slice (invisible keys give 0), row-sum accumulation in
+// packed fp32 pairs, and the bf16 pairs of P.
+__device__ __forceinline__ void exp_slice(uint32_t (&sr)[32], uint32_t vis, uint64_t sl2x2, uint64_t nm2,
+                                          uint64_t& acc0, uint64_t& acc1, uint32_t (&pk)[16]) {
+  if (vis != 0xffffffffu) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+      if (!((vis >> c) & 1u)) sr[c] = 0xff800000u;  // -inf
+  }
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    const uint64_t y = f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nm2);
+    float y0, y1;
+    f2_unpack(y, y0, y1);
+    const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+    if ((c >> 1) & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
+    else acc0 = f2_add(acc0, f2_pack(p0, p1));
+    pk[c >> 1] = pack_bf16x2(p0, p1);
+  }
+}
+
+__device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uint32_t tmem, int qt) {
+  const int r = threadIdx.x - 128 - qt * kBM;  // row of M tile qt == TMEM lane
   const int wq = (threadIdx.x >> 5) & 3;
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const uint32_t s_col = kTmS + qt * 128, o_col = kTmO + qt * 128;
   volatile int* abort = &s.abort_flag;
   const float sl2 = p.scale_log2;
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -462,39 +508,39 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
   uint32_t it = 0, sidx = 0;
   while (iter.next(s, p, g)) {
     const int buf = sidx & 1;
-    const int node = g.mt * nodes_per_tile + r / p.group;
+    const int node = (g.mp * kAttnQTiles + qt) * nodes_per_tile + r / p.group;
     const int head = g.kvh * p.group + (r % p.group);
     const bool row_valid = node < g.N;
     const uint32_t* anc = &s.anc[buf][row_valid ? node : 0][0];
     float m_use = -INFINITY, l = 0.f;
     bool meta_seen = false;
     for (int t = g.kb; t < g.ke; ++t, ++it) {
-      const int sb = it & 1;
       const bool tree_tile = (t + 1) * kBN > g.P;
       if (tree_tile && !meta_seen) {
         if (!warp_wait(&s.bar_metafull[buf], (sidx >> 1) & 1, abort)) return set_abort(s, p);
         meta_seen = true;
       }
-      if (!warp_wait(&s.bar_sfull[sb], (it >> 1) & 1, abort)) return set_abort(s, p);
-      // S(it) ready implies PV(it-2) is complete (the tensor pipe runs in issue order); observing that
-      // phase keeps pvdone[it & 1] in step so later waits on it are unambiguous.
-      if (it >= 2 && !warp_wait(&s.bar_pvdone[sb], ((it - 2) >> 1) & 1, abort)) return set_abort(s, p);
+      if (!warp_wait(&s.bar_sfull[qt], it & 1, abort)) return set_abort(s, p);
+      // S_qt(it) ready implies PV_qt(it-1) is complete (the tensor pipe runs in issue order); observing
+      // that phase keeps the pv-done barrier in step for the epilogue's wait.
+      if (it >= 1 && !warp_wait(&s.bar_pvdone[qt], (it - 1) & 1, abort)) return set_abort(s, p);
       tc_fence_after();
+      // the whole 128-column row of S in registers: one TMEM round trip per tile
       uint32_t sr[128];
-      tmem_ld32(lane_base + sb * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(lane_base + sb * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(lane_base + sb * 128 + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      tmem_ld32(lane_base + sb * 128 + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_ld32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(lane_base + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(lane_base + s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      uint32_t vis[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+        vis[w] = tree_tile ? vis_word(t * kBN + 32 * w, g.P, g.N, row_valid, anc) : 0xffffffffu;
       tmem_ld_wait();
       if (tree_tile) {
         // invisible keys become -inf: they drop out of the max and get P = 2^-inf = 0
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const uint32_t vw = vis_word(t * kBN + 32 * w, g.P, g.N, row_valid, anc);
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (!((vw >> i) & 1u)) sr[32 * w + i] = 0xff800000u;
-        }
+        for (int c = 0; c < 128; ++c)
+          if (!((vis[c >> 5] >> (c & 31)) & 1u)) sr[c] = 0xff800000u;
       }
       float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
@@ -518,59 +564,53 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
       }
       const float negm = (m_use == -INFINITY) ? 0.f : -m_use;
       const uint64_t nm2 = f2_pack(negm, negm);
-      uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;
-      uint32_t pk[64];
+      // P = 2^(s * scale - m), row sum in packed pairs, bf16 pairs of P written over S's first 64 columns
+      uint64_t acc0 = 0, acc1 = 0;
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const uint64_t y = f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nm2);
-        float y0, y1;
-        f2_unpack(y, y0, y1);
-        const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
-        const uint64_t pp = f2_pack(p0, p1);
-        switch ((c >> 1) & 3) {
-          case 0: acc0 = f2_add(acc0, pp); break;
-          case 1: acc1 = f2_add(acc1, pp); break;
-          case 2: acc2 = f2_add(acc2, pp); break;
-          default: acc3 = f2_add(acc3, pp); break;
+      for (int h = 0; h < 2; ++h) {  // two halves, so only 32 packed words are live at a time
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const int cc = 64 * h + c;
+          const uint64_t y = f2_fma(f2_pack(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), sl2x2, nm2);
+          float y0, y1;
+          f2_unpack(y, y0, y1);
+          const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+          if ((c >> 1) & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
+          else acc0 = f2_add(acc0, f2_pack(p0, p1));
+          pk[c >> 1] = pack_bf16x2_alu(p0, p1);
         }
-        pk[c >> 1] = pack_bf16x2(p0, p1);
+        tmem_st32(lane_base + s_col + 32 * h, pk);
       }
       {
-        const uint64_t t2 = f2_add(f2_add(acc0, acc1), f2_add(acc2, acc3));
-        float u0, u1;
-        f2_unpack(t2, u0, u1);
-        l += u0 + u1;
+        float u0, u1, v0, v1;
+        f2_unpack(acc0, u0, u1);
+        f2_unpack(acc1, v0, v1);
+        l += (u0 + u1) + (v0 + v1);
       }
       if (__any_sync(0xffffffffu, resc)) {
-        // O must hold PV(it-1) before it is rescaled
-        if (!warp_wait(&s.bar_pvdone[(it - 1) & 1], ((it - 1) >> 1) & 1, abort)) return set_abort(s, p);
-        tc_fence_after();
+        // O_qt already holds PV_qt(it-1) (implied by S_qt(it) being ready)
         const float a = resc ? alpha : 1.f;
 #pragma unroll
         for (int cc = 0; cc < 128; cc += 32) {
           uint32_t o[32];
-          tmem_ld32(lane_base + kTmO + cc, o);
+          tmem_ld32(lane_base + o_col + cc, o);
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * a);
-          tmem_st32(lane_base + kTmO + cc, o);
+          tmem_st32(lane_base + o_col + cc, o);
         }
       }
-      tmem_st32(lane_base + sb * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(lane_base + sb * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&s.bar_pfull[sb]);
+      mbar_arrive(&s.bar_pfull[qt]);
     }
     // ---------------- epilogue of the segment
     if (!meta_seen) {
       if (!warp_wait(&s.bar_metafull[buf], (sidx >> 1) & 1, abort)) return set_abort(s, p);
     }
     const bool seg_ok = s.meta_valid[buf] != 0;
-    {
-      const uint32_t last = it - 1;
-      if (!warp_wait(&s.bar_pvdone[last & 1], (last >> 1) & 1, abort)) return set_abort(s, p);
-    }
+    if (!warp_wait(&s.bar_pvdone[qt], (it - 1) & 1, abort)) return set_abort(s, p);
     tc_fence_after();
     mbar_arrive(&s.bar_metaempty[buf]);
     const bool split = g.c0 != g.c1;
@@ -580,98 +620,37 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
 #pragma unroll
       for (int cc = 0; cc < 128; cc += 32) {
         uint32_t o[32];
-        tmem_ld32(lane_base + kTmO + cc, o);
+        tmem_ld32(lane_base + o_col + cc, o);
         tmem_ld_wait();
         if (seg_ok && row_valid)
           store_row_bf16(p.out + grow * 128 + cc, reinterpret_cast<const float*>(o), inv_l);
       }
       if (seg_ok && row_valid && p.lse != nullptr) p.lse[grow] = (m_use + __log2f(l)) * 0.69314718055994531f;
     } else {
+      // unit cut between CTAs: store this segment's unnormalised O, (m, l) and validity; the combine
+      // kernel that runs after this one merges the segments
+      const int myslot = g.slot * kAttnQTiles + qt;
 #pragma unroll
       for (int cc = 0; cc < 128; cc += 32) {
         uint32_t o[32];
-        tmem_ld32(lane_base + kTmO + cc, o);
+        tmem_ld32(lane_base + o_col + cc, o);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 32; c += 4)
-          __stcg(part_ptr(p, g.slot, (cc + c) >> 2, r),
+          __stcg(part_ptr(p, myslot, (cc + c) >> 2, r),
                  make_float4(__uint_as_float(o[c]), __uint_as_float(o[c + 1]), __uint_as_float(o[c + 2]),
                              __uint_as_float(o[c + 3])));
       }
-      __stcg(&p.part_ml[static_cast<long long>(g.slot) * kBM + r], make_float2(m_use, l));
-      __stcg(&p.part_ok[static_cast<long long>(g.slot) * kBM + r], seg_ok ? 1 : 0);
-      __threadfence();
-      int* ctr = p.counters + static_cast<long long>(g.c0) * kBM + r;
-      const int prev = atomicAdd(ctr, 1);
-      if (prev == g.c1 - g.c0) {
-        // last contributor for this row: merge every CTA's partial; loads are issued four segments and
-        // 32 columns at a time so each batch is one memory round trip
-        __threadfence();
-        constexpr int kGrp = 4;
-        float M = -INFINITY, L = 0.f;
-        bool all_ok = true;
-        for (int cb = g.c0; cb <= g.c1; cb += kGrp) {
-          float2 ml[kGrp];
-          int ok[kGrp];
-#pragma unroll
-          for (int u = 0; u < kGrp; ++u) {
-            const int c = cb + u;
-            const int sl = (c == g.c0) ? 2 * c + 1 : 2 * c;
-            ml[u] = c <= g.c1 ? __ldcg(&p.part_ml[static_cast<long long>(sl) * kBM + r]) : make_float2(-INFINITY, 0.f);
-            ok[u] = c <= g.c1 ? __ldcg(&p.part_ok[static_cast<long long>(sl) * kBM + r]) : 1;
-          }
-#pragma unroll
-          for (int u = 0; u < kGrp; ++u) {
-            M = fmaxf(M, ml[u].x);
-            all_ok = all_ok && ok[u] != 0;
-          }
-        }
-        for (int cb = g.c0; cb <= g.c1; cb += kGrp) {
-#pragma unroll
-          for (int u = 0; u < kGrp; ++u) {
-            const int c = cb + u;
-            const int sl = (c == g.c0) ? 2 * c + 1 : 2 * c;
-            if (c <= g.c1) {
-              const float2 ml = __ldcg(&p.part_ml[static_cast<long long>(sl) * kBM + r]);
-              if (ml.x != -INFINITY) L += ml.y * ex2_approx(ml.x - M);
-            }
-          }
-        }
-        const float inv_L = 1.f / L;
-        for (int cc = 0; cc < 128; cc += 32) {
-          float acc[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) acc[c] = 0.f;
-          for (int cb = g.c0; cb <= g.c1; cb += kGrp) {
-            float4 v[kGrp][8];
-            float w[kGrp];
-#pragma unroll
-            for (int u = 0; u < kGrp; ++u) {
-              const int c = cb + u;
-              const int sl = (c == g.c0) ? 2 * c + 1 : 2 * c;
-              const bool have = c <= g.c1;
-              const float2 ml = have ? __ldcg(&p.part_ml[static_cast<long long>(sl) * kBM + r])
-                                     : make_float2(-INFINITY, 0.f);
-              w[u] = (ml.x == -INFINITY) ? 0.f : ex2_approx(ml.x - M);
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                v[u][q] = have ? __ldcg(part_ptr(p, sl, (cc >> 2) + q, r)) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < kGrp; ++u) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                acc[4 * q + 0] = fmaf(w[u], v[u][q].x, acc[4 * q + 0]);
-                acc[4 * q + 1] = fmaf(w[u], v[u][q].y, acc[4 * q + 1]);
-                acc[4 * q + 2] = fmaf(w[u], v[u][q].z, acc[4 * q + 2]);
-                acc[4 * q + 3] = fmaf(w[u], v[u][q].w, acc[4 * q + 3]);
-              }
-            }
-          }
-          if (all_ok && row_valid) store_row_bf16(p.out + grow * 128 + cc, acc, inv_L);
-        }
-        if (all_ok && row_valid && p.lse != nullptr) p.lse[grow] = (M + __log2f(L)) * 0.69314718055994531f;
-        *ctr = 0;  // leave the workspace zeroed for the next call
+      __stcg(&p.part_ml[static_cast<long long>(myslot) * kBM + r], make_float2(m_use, l));
+      __stcg(&p.part_ok[static_cast<long long>(myslot) * kBM + r], seg_ok ? 1 : 0);
+      if (static_cast<int>(blockIdx.x) == g.c0 && r == 0) {
+        // descriptor of the split unit, indexed by its first CTA (unique per split unit)
+        int4 d;
+        d.x = g.c1;
+        d.y = g.off + g.mp * kAttnQTiles * nodes_per_tile;  // first global node of the unit
+        d.z = g.N - g.mp * kAttnQTiles * nodes_per_tile;    // nodes of the sequence from there on
+        d.w = g.kvh;
+        if (qt == 0) __stcg(&p.units[g.c0], d);
       }
     }
     ++sidx;
@@ -684,6 +663,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5;
+  // Slot blockIdx.x of the split-unit table is written only by this CTA (if it starts a split unit);
+  // clear what an earlier call left there before anything else.
+  if (tid == 0 && blockIdx.x < kMaxGrid) p.units[blockIdx.x] = make_int4(0, 0, 0, 0);
+  // Let the combine kernel be scheduled now; its griddepcontrol.wait still holds it until this grid
+  // has finished, but it no longer pays a launch after the last CTA exits.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   build_plan(s, p);
   if (s.bad_meta) {
@@ -718,12 +703,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.bar_vfull[i], 1);
       mbar_init(&s.bar_vempty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAttnQTiles; ++i) {
       mbar_init(&s.bar_sfull[i], 1);
-      mbar_init(&s.bar_pfull[i], 128);
-      mbar_init(&s.bar_metafull[i], 32);
-      mbar_init(&s.bar_metaempty[i], 128);
+      mbar_init(&s.bar_pfull[i], kBM);
       mbar_init(&s.bar_pvdone[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.bar_metafull[i], 32);
+      mbar_init(&s.bar_metaempty[i], kAttnQTiles * kBM);
     }
     s.abort_flag = 0;
     fence_barrier_init();
@@ -742,14 +729,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  if (warp == 0 || warp == 2) {
-    kv_producer(s, p, iter, warp == 2, &tm_q, warp == 2 ? &tm_v : &tm_k);
-  } else if (warp == 1) {
-    mma_issuer(s, p, iter, tmem);
-  } else if (warp == 3) {
-    metadata(s, p, iter);
+  // Register split (the launch gives every thread 168): the copy/MMA/metadata warpgroup runs on 64,
+  // which lets the two softmax warpgroups hold a whole 128-column row of S in registers (208).
+  // 128 * 64 + 256 * 208 = 61440 <= 384 * 168 = 64512 (the launch's register pool).
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
+    if (warp == 0 || warp == 2) {
+      kv_producer(s, p, iter, warp == 2, &tm_q, warp == 2 ? &tm_v : &tm_k);
+    } else if (warp == 1) {
+      mma_issuer(s, p, iter, tmem);
+    } else {
+      metadata(s, p, iter);
+    }
   } else {
-    softmax_epilogue(s, p, iter, tmem);
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
+    softmax_epilogue(s, p, iter, tmem, warp < 8 ? 0 : 1);
   }
   tc_fence_before();
   __syncthreads();
@@ -759,22 +753,125 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// Combine kernel: merges the partials of every unit that was cut between CTAs.  Block (c0, q, rb)
+// handles rows [32 rb, 32 rb + 32) of M tile q of the unit whose first CTA is c0; each of its 256
+// threads owns one row and four 4-column groups and loads the unit's segments four at a time (a unit
+// cut into at most four pieces is merged in one memory round trip).
+// Launched right after the attention kernel (programmatic dependent launch), it waits for the
+// attention grid before reading.
+// ------------------------------------------------------------------------------------------------
+constexpr int kCombineRows = 32;
+constexpr int kCombineQuads = 4;  // 4-column groups per thread
+constexpr int kSegBatch = 4;      // segments whose partials are loaded in one batch
+
+__global__ void __launch_bounds__(256, 2) combine_kernel(const AttnParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the attention grid has completed
+  const int c0 = blockIdx.x;
+  const int qt = blockIdx.y;
+  const int rb = blockIdx.z;
+  const int4 d = __ldcg(&p.units[c0]);
+  const int c1 = d.x;
+  if (c1 <= c0) return;  // no split unit starts at this CTA
+  const int rl = threadIdx.x & (kCombineRows - 1);
+  const int q0 = (threadIdx.x >> 5) * kCombineQuads;  // first 4-column group of this thread
+  const int r = rb * kCombineRows + rl;               // row of the M tile
+  const int nodes_per_tile = kBM / p.group;
+  const int node = qt * nodes_per_tile + r / p.group;
+  if (node >= d.z) return;
+  const long long grow = static_cast<long long>(d.y + node) * p.hq + d.w * p.group + (r % p.group);
+  float M = -INFINITY;
+  bool ok = true;
+  for (int cb = c0; cb <= c1; cb += kSegBatch) {
+#pragma unroll
+    for (int u = 0; u < kSegBatch; ++u) {
+      const int c = cb + u;
+      if (c <= c1) {
+        const int sl = slot_of(c, c0) * kAttnQTiles + qt;
+        M = fmaxf(M, __ldcg(&p.part_ml[static_cast<long long>(sl) * kBM + r]).x);
+        ok = ok && __ldcg(&p.part_ok[static_cast<long long>(sl) * kBM + r]) != 0;
+      }
+    }
+  }
+  float L = 0.f;
+  float4 acc[kCombineQuads];
+#pragma unroll
+  for (int q = 0; q < kCombineQuads; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int cb = c0; cb <= c1; cb += kSegBatch) {
+    float2 ml[kSegBatch];
+    float4 v[kSegBatch][kCombineQuads];
+#pragma unroll
+    for (int u = 0; u < kSegBatch; ++u) {
+      const int c = cb + u;
+      const int sl = slot_of(c, c0) * kAttnQTiles + qt;
+      const bool have = c <= c1;
+      ml[u] = have ? __ldcg(&p.part_ml[static_cast<long long>(sl) * kBM + r]) : make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int q = 0; q < kCombineQuads; ++q)
+        v[u][q] = have ? __ldcg(part_ptr(p, sl, q0 + q, r)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kSegBatch; ++u) {
+      if (ml[u].x == -INFINITY) continue;
+      const float w = ex2_approx(ml[u].x - M);
+      L = fmaf(w, ml[u].y, L);
+#pragma unroll
+      for (int q = 0; q < kCombineQuads; ++q) {
+        acc[q].x = fmaf(w, v[u][q].x, acc[q].x);
+        acc[q].y = fmaf(w, v[u][q].y, acc[q].y);
+        acc[q].z = fmaf(w, v[u][q].z, acc[q].z);
+        acc[q].w = fmaf(w, v[u][q].w, acc[q].w);
+      }
+    }
+  }
+  if (!ok) return;
+  const float inv = 1.f / L;
+  uint4 o[2];
+  o[0].x = pack_bf16x2(acc[0].x * inv, acc[0].y * inv);
+  o[0].y = pack_bf16x2(acc[0].z * inv, acc[0].w * inv);
+  o[0].z = pack_bf16x2(acc[1].x * inv, acc[1].y * inv);
+  o[0].w = pack_bf16x2(acc[1].z * inv, acc[1].w * inv);
+  o[1].x = pack_bf16x2(acc[2].x * inv, acc[2].y * inv);
+  o[1].y = pack_bf16x2(acc[2].z * inv, acc[2].w * inv);
+  o[1].z = pack_bf16x2(acc[3].x * inv, acc[3].y * inv);
+  o[1].w = pack_bf16x2(acc[3].z * inv, acc[3].w * inv);
+  uint4* dst = reinterpret_cast<uint4*>(p.out + grow * 128 + q0 * 4);
+  dst[0] = o[0];
+  dst[1] = o[1];
+  if (q0 == 0 && p.lse != nullptr) p.lse[grow] = (M + __log2f(L)) * 0.69314718055994531f;
+}
+
 }  // namespace attn
 
 size_t attention_smem_bytes() { return sizeof(attn::Smem) + 1024; }
 
 cudaError_t launch_tree_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                   const AttnParams& p, int grid, cudaStream_t stream) {
-  static bool attr_set = false;
+  static std::atomic<bool> attr_set[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
   const size_t smem = attention_smem_bytes();
-  if (!attr_set) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(attn::tree_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   attn::tree_attention_kernel<<<grid, attn::kThreads, smem, stream>>>(tm_q, tm_k, tm_v, p);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // The combine kernel may start as soon as the attention grid is scheduled; its griddepcontrol.wait
+  // holds it until the attention grid has finished and its writes are visible.
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, kAttnQTiles, kAttnRows / attn::kCombineRows);
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn::combine_kernel, p);
 }
 
 }  // namespace jf
