@@ -69,6 +69,16 @@ def make_inputs(cfg, seed):
                 offsets=(np.arange(B + 1) * N).astype(np.int32))
 
 
+def rank_seed(rank):
+    """Every rank verifies its own independent seeded batch (weak scaling)."""
+    return 1000 + rank
+
+
+def job_nodes_per_sec(batch, budget, world, step_ms):
+    """Whole-job throughput: all ranks' tree nodes over the max-over-ranks step time."""
+    return batch * budget * world / (step_ms * 1e-3)
+
+
 def visible_pairs(parent, prefix):
     """sum over nodes of |visible set| = P + depth(node) (node with parent -1 has depth 1)."""
     tot = 0
@@ -169,7 +179,7 @@ def run_gpu(args, cfg, rank, world, device):
     from tree_verify_attention_jf_b200 import api, synth
 
     torch.cuda.set_device(device)
-    seed = 1000 + rank
+    seed = rank_seed(rank)
     inp = make_inputs(cfg, seed)
     B, N, V = cfg["batch"], cfg["budget"], cfg["vocab"]
     gen = torch.Generator(device=device).manual_seed(seed)
@@ -329,7 +339,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        rate, steps, el, threads = oracle_step_rate(cfg, 1000)
+        rate, steps, el, threads = oracle_step_rate(cfg, rank_seed(0))
         line = {"impl": "reference", "metric": metric, "value": rate, "unit": "nodes/s", "n_gpus": args.gpus,
                 "steps": steps, "warmup": 0, "ms_per_step": 1e3 * el / steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
@@ -352,7 +362,6 @@ def main():
     e2e_step = max_over_ranks(statistics.mean(r["e2e_ms"]), world, device)
     attn_ms = statistics.mean(r["attn_ms"])
     B, N = cfg["batch"], cfg["budget"]
-    nodes = B * N * world
     pk = peaks()
     pairs = visible_pairs(r["parent"], [cfg["prefix"]] * B)
     flops = 4.0 * HEAD_DIM * cfg["hq"] * pairs
@@ -370,11 +379,11 @@ def main():
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        rate, steps, el, threads = oracle_step_rate(cfg, 1000)
+        rate, steps, el, threads = oracle_step_rate(cfg, rank_seed(0))
         cpu = {"value": rate, "unit": "nodes/s", "cores": threads, "kind": "oracle",
                "sample": f"{steps} whole step(s) of the same workload (build + attention + accept), {el:.1f} s"}
     line = {
-        "metric": metric, "value": nodes / (step_ms * 1e-3), "unit": "nodes/s", "n_gpus": world, "steps": args.steps,
+        "metric": metric, "value": job_nodes_per_sec(B, N, world, step_ms), "unit": "nodes/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)", "config": config,
         "roofline": {"kernel": "jf::attn::tree_attention_kernel", "bound": "tensor", "achieved": tflops,
@@ -385,7 +394,7 @@ def main():
         "kernel_ms": {"build_tree": statistics.mean(r["build_ms"]), "tree_attention": attn_ms,
                       "accept": statistics.mean(r["accept_ms"])},
         "time_share": shares,
-        "e2e": {"value": nodes / (e2e_step * 1e-3), "unit": "nodes/s", "h2d_bytes_per_step": r["h2d"],
+        "e2e": {"value": job_nodes_per_sec(B, N, world, e2e_step), "unit": "nodes/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         # per step: row statistics + best-first expansion, attention + split combine, accept
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,

@@ -22,8 +22,10 @@
 //     of O, and the epilogue.
 //   * The tree mask only touches tiles that hold tree slots; prefix tiles are unmasked.
 //   * Work split: the flattened (unit, kv tile) space is cut into equal contiguous ranges, one per CTA
-//     (stream-K).  A unit cut between CTAs writes fp32 partials; per row, the last CTA to finish (an
-//     atomic counter per row, no spinning) merges them and stores the bf16 output.
+//     (stream-K).  A unit cut between CTAs writes fp32 partials (O, running max, row sum) and its
+//     first CTA records the unit in a descriptor slot; combine_kernel, launched right behind on the
+//     same stream with a programmatic dependency, merges each recorded unit's partials and stores the
+//     bf16 output.  Nothing spins on another CTA.
 #include "jf_device.cuh"
 #include "jf_internal.h"
 
@@ -42,12 +44,17 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmS = 0;    // S_i at column 128 * i
 constexpr uint32_t kTmO = 256;  // O_i at column 256 + 128 * i
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow up to 2^8 before O is rescaled
+// Pairs of P (bit i: columns 2i, 2i+1 of each 64-column half) whose 2^y is evaluated on the FMA pipe
+// by a polynomial instead of by MUFU ex2: the two softmax warpgroups share each SM's 16 ex2 per
+// clock, and moving part of the work to the otherwise idle FMA pipe shortens the exp phase.
+constexpr uint32_t kPolyPairs = 0x00000000u;
 
 struct __align__(1024) Smem {
   uint8_t q[kAttnQTiles][kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
   uint32_t anc[2][kMaxTreeNodes][kAncWords];
+  int par_stage[kMaxTreeNodes];  // the metadata warp's copy of the current segment's parent indices
   long long cum_work[kMaxAttnBatch + 1];
   long long scan_warp[kThreads / 32];
   uint64_t bar_qfull, bar_qempty;
@@ -339,28 +346,43 @@ __device__ void metadata(Smem& s, const AttnParams& p, SegIter iter) {
     }
     __syncwarp();
     if (s.meta_ctl == 0) return;
-    // --- validation: parent indices, capacity, the page ids this segment reads
-    int bad = 0;
+    // --- validation: parent indices, capacity, the page ids this segment reads.  Every global load of
+    // the segment is issued before any is used, so the whole check costs one memory round trip.
     const int npg = (g.P + g.N + kPage - 1) / kPage;
-    if (static_cast<long long>(g.P) + g.N > static_cast<long long>(p.max_pages) * kPage) bad = 1;
     const int32_t* par = p.parent + g.off;
-    for (int i = lane; i < g.N; i += 32) {
-      const int pi = par[i];
-      if (pi < -1 || pi >= i) bad = 1;
-    }
     const int32_t* bt = p.block_table + static_cast<long long>(g.b) * p.max_pages;
+    int pr[kMaxTreeNodes / 32];
+#pragma unroll
+    for (int k = 0; k < kMaxTreeNodes / 32; ++k) {
+      const int i = lane + 32 * k;
+      pr[k] = i < g.N ? __ldg(par + i) : -1;
+    }
     int pg1 = g.ke * kPagesPerTile;
     if (pg1 > npg) pg1 = npg;
     if (pg1 > p.max_pages) pg1 = p.max_pages;
-    for (int pg = g.kb * kPagesPerTile + lane; pg < pg1; pg += 32) {
-      const int v = bt[pg];
-      if (v < 0 || v >= p.num_pages) bad = 1;
+    int bad = (static_cast<long long>(g.P) + g.N > static_cast<long long>(p.max_pages) * kPage) ? 1 : 0;
+    for (int pg = g.kb * kPagesPerTile + lane; pg < pg1; pg += 4 * 32) {
+      int v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = (pg + 32 * u < pg1) ? __ldg(bt + pg + 32 * u) : 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v[u] < 0 || v[u] >= p.num_pages) bad = 1;
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxTreeNodes / 32; ++k) {
+      const int i = lane + 32 * k;
+      if (i < g.N) {
+        if (pr[k] < -1 || pr[k] >= i) bad = 1;
+        s.par_stage[i] = (pr[k] >= i) ? -1 : pr[k];  // invalid parents are flagged; keep the walk in range
+      }
     }
     bad = __any_sync(0xffffffffu, bad);
     if (lane == 0) {
       s.meta_valid[buf] = bad ? 0 : 1;
       if (bad) report(p.status, JF_ERR_DEVICE_CHECK);
     }
+    __syncwarp();
     // --- ancestor bitsets (only needed when the segment reaches the tree slots).  Nodes are taken
     // 32 at a time in index order; a node whose parent lies in an earlier chunk starts from the
     // parent's finished bitset, the others resolve their in-chunk chain by pointer jumping over warp
@@ -374,8 +396,7 @@ __device__ void metadata(Smem& s, const AttnParams& p, SegIter iter) {
         int jl = -1;  // lane of the next in-chunk ancestor still to merge
         if (i < g.N) {
           a[i >> 5] = 1u << (i & 31);
-          int pi = par[i];
-          if (pi >= i) pi = -1;  // invalid parents were flagged above; keep the walk in range
+          const int pi = s.par_stage[i];
           if (pi >= 0 && pi < base) {
 #pragma unroll
             for (int w = 0; w < kAncWords; ++w) a[w] |= s.anc[buf][pi][w];
@@ -456,45 +477,6 @@ __device__ __forceinline__ float4* part_ptr(const AttnParams& p, int slot, int c
   return reinterpret_cast<float4*>(p.part_o) + (static_cast<long long>(slot) * 32 + c4) * kBM + r;
 }
 
-__device__ __forceinline__ float slice_max(const uint32_t (&sr)[32], uint32_t vis) {
-  float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
-  if (vis == 0xffffffffu) {
-#pragma unroll
-    for (int c = 0; c < 32; c += 8) {
-      a0 = fmax3(a0, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
-      a1 = fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-      a2 = fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-      a3 = fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < 32; ++c)
-      if ((vis >> c) & 1u) a0 = fmaxf(a0, __uint_as_float(sr[c]));
-  }
-  return fmax3(a0, a1, fmaxf(a2, a3));
-}
-
-// P = 2^(s * scale - m) for one 32-column slice (invisible keys give 0), row-sum accumulation in
-// packed fp32 pairs, and the bf16 pairs of P.
-__device__ __forceinline__ void exp_slice(uint32_t (&sr)[32], uint32_t vis, uint64_t sl2x2, uint64_t nm2,
-                                          uint64_t& acc0, uint64_t& acc1, uint32_t (&pk)[16]) {
-  if (vis != 0xffffffffu) {
-#pragma unroll
-    for (int c = 0; c < 32; ++c)
-      if (!((vis >> c) & 1u)) sr[c] = 0xff800000u;  // -inf
-  }
-#pragma unroll
-  for (int c = 0; c < 32; c += 2) {
-    const uint64_t y = f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nm2);
-    float y0, y1;
-    f2_unpack(y, y0, y1);
-    const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
-    if ((c >> 1) & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
-    else acc0 = f2_add(acc0, f2_pack(p0, p1));
-    pk[c >> 1] = pack_bf16x2(p0, p1);
-  }
-}
-
 __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uint32_t tmem, int qt) {
   const int r = threadIdx.x - 128 - qt * kBM;  // row of M tile qt == TMEM lane
   const int wq = (threadIdx.x >> 5) & 3;
@@ -573,9 +555,15 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
         for (int c = 0; c < 64; c += 2) {
           const int cc = 64 * h + c;
           const uint64_t y = f2_fma(f2_pack(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), sl2x2, nm2);
-          float y0, y1;
-          f2_unpack(y, y0, y1);
-          const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+          float p0, p1;
+          if ((kPolyPairs >> (c >> 1)) & 1u) {
+            exp2_poly2(y, p0, p1);
+          } else {
+            float y0, y1;
+            f2_unpack(y, y0, y1);
+            p0 = ex2_approx(y0);
+            p1 = ex2_approx(y1);
+          }
           if ((c >> 1) & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
           else acc0 = f2_add(acc0, f2_pack(p0, p1));
           pk[c >> 1] = pack_bf16x2_alu(p0, p1);
@@ -729,11 +717,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  // Register split (the launch gives every thread 168): the copy/MMA/metadata warpgroup runs on 64,
+  // Register split (the launch gives every thread 168): the copy/MMA/metadata warpgroup runs on 80,
   // which lets the two softmax warpgroups hold a whole 128-column row of S in registers (208).
-  // 128 * 64 + 256 * 208 = 61440 <= 384 * 168 = 64512 (the launch's register pool).
+  // 128 * 80 + 256 * 208 = 63488 <= 384 * 168 = 64512 (the launch's register pool).
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
     if (warp == 0 || warp == 2) {
       kv_producer(s, p, iter, warp == 2, &tm_q, warp == 2 ? &tm_v : &tm_k);
     } else if (warp == 1) {
