@@ -9,9 +9,10 @@
 // than bandwidth.  Each sequence gets one thread-block cluster (16 CTAs where the GPU allows it,
 // else 8); every CTA reduces its slice of the current row with 16-byte loads issued eight deep, the
 // partial (value, id) pairs are exchanged through distributed shared memory, and every CTA derives
-// the same next node.  While a row is being reduced, the rows of the
-// current node's children (the only candidates for the next step) are prefetched into L2 with bulk
-// prefetches, so the next step reads from L2.
+// the same next node, with one cluster barrier per step.  The children of every node are listed
+// once at the start; while a row is being reduced, the rows of the current node's children (the
+// only candidates for the next step) are prefetched into L2 with bulk prefetches, so the next step
+// reads from L2.
 #include <cooperative_groups.h>
 
 #include "jf_device.cuh"
@@ -55,6 +56,17 @@ __device__ __forceinline__ void prefetch_l2(const float* p, long long n) {
   }
 }
 
+__device__ __forceinline__ void warp_best(float& v, int& id) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, v, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, id, off);
+    take(ov, oi, v, id);
+  }
+}
+
+constexpr int kWarps = kThreads / 32;
+
 __global__ void __launch_bounds__(kThreads)
     accept_kernel(const int32_t* __restrict__ token, const int32_t* __restrict__ parent,
                   const float* __restrict__ logits, int num_nodes, int vocab, int max_depth,
@@ -62,11 +74,15 @@ __global__ void __launch_bounds__(kThreads)
                   int32_t* __restrict__ status) {
   __shared__ int s_tok[kMaxAcceptNodes];
   __shared__ int s_par[kMaxAcceptNodes];
+  __shared__ int s_cur[kMaxAcceptNodes];      // children per node, then the fill cursor
+  __shared__ int s_off[kMaxAcceptNodes + 1];  // children of node n: s_kid[s_off[n] .. s_off[n + 1])
+  __shared__ int s_kid[kMaxAcceptNodes];
   __shared__ int s_path[kMaxAcceptNodes + 1];
-  __shared__ Best s_slot[2];  // this CTA's partial argmax, double-buffered across steps
-  __shared__ Best s_warp[kThreads / 32];
-  __shared__ int s_kids[kMaxAcceptNodes];
-  __shared__ int s_nkids, s_match, s_arg, s_bad;
+  __shared__ Best s_part[kWarps];  // this step's per-warp partial argmax
+  __shared__ Best s_slot[2];       // this CTA's partial argmax, by step parity (read by the whole cluster)
+  __shared__ int2 s_dec[2];        // (argmax, next node) of the step, by step parity
+  __shared__ int s_wsum[kWarps];
+  __shared__ int s_bad;
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
@@ -75,44 +91,66 @@ __global__ void __launch_bounds__(kThreads)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t* tk = token + static_cast<long long>(b) * num_nodes;
   const int32_t* pr = parent + static_cast<long long>(b) * num_nodes;
-  if (tid == 0) s_bad = 0;
-  __syncthreads();
-  for (int i = tid; i < num_nodes; i += kThreads) {
-    const int pi = pr[i];
-    s_par[i] = pi;
-    s_tok[i] = tk[i];
-    if (pi < -1 || pi >= i) s_bad = 1;
-  }
-  __syncthreads();
-  if (s_bad) {  // every CTA of the cluster sees the same data and leaves here together
-    if (rank == 0 && tid == 0) report(status, JF_ERR_DEVICE_CHECK);
-    return;
-  }
   // this CTA's slice of every row (a multiple of 4 entries, so 16-byte loads stay aligned)
   const int per = ((vocab + C - 1) / C + 3) & ~3;
   const int lo = min(vocab, rank * per);
   const int hi = min(vocab, lo + per);
   const float* rows = logits + static_cast<long long>(b) * num_nodes * vocab;
   const bool vec = (vocab % 4) == 0;  // rows then start 16-byte aligned (the base is checked on the host)
-
+  if (tid == 0 && hi > lo) prefetch_l2(rows + lo, hi - lo);  // the root's row, while the tree is read
+  // ---- the tree: tokens, parents (validated) and a children list per node
+  if (tid == 0) s_bad = 0;
+  for (int i = tid; i < num_nodes; i += kThreads) s_cur[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < num_nodes; i += kThreads) {
+    const int pi = pr[i];
+    s_par[i] = pi;
+    s_tok[i] = tk[i];
+    if (pi < -1 || pi >= i) s_bad = 1;
+    else if (pi >= 0) atomicAdd(&s_cur[pi], 1);
+  }
+  __syncthreads();
+  if (s_bad) {  // every CTA of the cluster sees the same data and leaves here together
+    if (rank == 0 && tid == 0) report(status, JF_ERR_DEVICE_CHECK);
+    return;
+  }
+  {
+    // exclusive prefix sum of the child counts (two entries per thread, num_nodes <= 2 * kThreads)
+    const int i0 = 2 * tid, i1 = 2 * tid + 1;
+    const int c0 = i0 < num_nodes ? s_cur[i0] : 0;
+    const int c1 = i1 < num_nodes ? s_cur[i1] : 0;
+    int incl = c0 + c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += s_wsum[w];
+    const int excl = base + incl - (c0 + c1);
+    if (i0 < num_nodes) s_off[i0] = excl;
+    if (i1 < num_nodes) s_off[i1] = excl + c0;
+    if (tid == kThreads - 1) s_off[num_nodes] = base + incl;
+    __syncthreads();
+    for (int i = tid; i < num_nodes; i += kThreads) s_cur[i] = s_off[i];
+    __syncthreads();
+    for (int i = tid; i < num_nodes; i += kThreads) {
+      const int pi = s_par[i];
+      if (pi >= 0) s_kid[atomicAdd(&s_cur[pi], 1)] = i;
+    }
+    __syncthreads();
+  }
+  // ---- the walk: per step one cluster barrier (partials visible cluster-wide) and two block barriers.
   int cur = 0, L = 0, a = 0;
   if (tid == 0) s_path[0] = 0;
   for (int step = 0;; ++step) {
     const float* row = rows + static_cast<long long>(cur) * vocab;
-    // children of cur: the candidates for the next row; prefetch their slices into L2
-    if (tid == 0) {
-      s_nkids = 0;
-      s_match = INT_MAX;
-    }
-    __syncthreads();
-    for (int c = tid; c < num_nodes; c += kThreads) {
-      if (s_par[c] == cur) s_kids[atomicAdd(&s_nkids, 1)] = c;
-    }
-    __syncthreads();
-    const int nk = s_nkids;
-    if (L < max_depth && tid < nk && hi > lo) {
-      prefetch_l2(rows + static_cast<long long>(s_kids[tid]) * vocab + lo, hi - lo);
-    }
+    const int k0 = s_off[cur], nk = s_off[cur + 1] - k0;
+    // the children of cur are the only candidates for the next row: prefetch their slices into L2
+    if (L < max_depth && tid < nk && hi > lo)
+      prefetch_l2(rows + static_cast<long long>(s_kid[k0 + tid]) * vocab + lo, hi - lo);
     // argmax of row cur over [lo, hi): lowest id among equal maxima
     float bv = -INFINITY;
     int bid = INT_MAX;
@@ -147,65 +185,48 @@ __global__ void __launch_bounds__(kThreads)
         for (int u = 0; u < kUnroll; ++u) take(v[u], base + u * kThreads, bv, bid);
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bid, off);
-      take(ov, oi, bv, bid);
-    }
-    if (lane == 0) s_warp[warp] = Best{bv, bid};
+    warp_best(bv, bid);
+    if (lane == 0) s_part[warp] = Best{bv, bid};
     __syncthreads();
     if (warp == 0) {
-      Best m = lane < kThreads / 32 ? s_warp[lane] : Best{-INFINITY, INT_MAX};
-#pragma unroll
-      for (int off = 8; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, m.v, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, m.id, off);
-        take(ov, oi, m.v, m.id);
-      }
+      Best m = lane < kWarps ? s_part[lane] : Best{-INFINITY, INT_MAX};
+      warp_best(m.v, m.id);
       if (lane == 0) s_slot[step & 1] = m;
     }
     cluster.sync();
-    // every CTA combines the partials of the whole cluster the same way
     if (warp == 0) {
+      // one warp per CTA gathers the cluster's partials and decides the next node
       Best m{-INFINITY, INT_MAX};
       if (lane < C) m = *cluster.map_shared_rank(&s_slot[step & 1], lane);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, m.v, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, m.id, off);
-        take(ov, oi, m.v, m.id);
-      }
-      if (lane == 0) {
-        int av = m.id;
-        if (av < 0 || av >= vocab) av = 0;  // only reachable with NaN rows
-        int match = INT_MAX;
-        if (L < max_depth) {
-          for (int k = 0; k < nk; ++k) {
-            const int c = s_kids[k];
-            if (s_tok[c] == av && c < match) match = c;
-          }
+      warp_best(m.v, m.id);
+      const int av = (m.id < 0 || m.id >= vocab) ? 0 : m.id;  // out of range only with NaN rows
+      // the child of cur carrying token av (the lowest index if several do)
+      int mt = INT_MAX;
+      if (L < max_depth) {
+        for (int k = lane; k < nk; k += 32) {
+          const int c = s_kid[k0 + k];
+          if (s_tok[c] == av && c < mt) mt = c;
         }
-        s_match = match;
-        s_arg = av;
       }
+      mt = __reduce_min_sync(0xffffffffu, mt);
+      if (lane == 0) s_dec[step & 1] = make_int2(av, mt);
     }
     __syncthreads();
-    a = s_arg;
-    const int match = s_match;
-    __syncthreads();  // everyone has read s_arg / s_match before they are reset
+    const int2 dec = s_dec[step & 1];
+    a = dec.x;
+    const int match = dec.y;
     if (match == INT_MAX) break;
     ++L;
     cur = match;
     if (tid == 0) s_path[L] = cur;
   }
-  if (rank == 0 && tid == 0) {
-    accepted_len[b] = L;
-    bonus[b] = a;
-  }
   if (rank == 0) {
-    int32_t* po = path + static_cast<long long>(b) * (max_depth + 1);
+    if (tid == 0) {
+      accepted_len[b] = L;
+      bonus[b] = a;
+    }
     __syncthreads();
+    int32_t* po = path + static_cast<long long>(b) * (max_depth + 1);
     for (int i = tid; i <= max_depth; i += kThreads) po[i] = (i <= L) ? s_path[i] : -1;
   }
   // keep every CTA's shared memory alive until the last remote read of it has happened

@@ -206,23 +206,23 @@ struct ExpandSmem {
   double key[kMaxBudget];  // sequential fallback: node keys
   int nsd[kMaxBudget];     // sequential fallback: next node of the same depth, in pop order
   int tail[kMaxDepths + 1];
-  int n_kept, n_surv;
 };
 
 // Level-parallel selection state (dynamic shared memory).  Nodes are kept in a pool in creation
-// order; lists hold pool ids.
+// order; lists hold pool ids.  The depth lists are double-buffered: the survivors of depth d (a prefix
+// of its list) are the parents of depth d + 1.
 constexpr int kPool = 4096;
+constexpr int kExpandThreads = 512;
 struct SelectSmem {
   double pool_key[kPool];
   int pool_par[kPool];  // parent's pool id, -1 = the root
   int pool_dr[kPool];   // (depth << 8) | rank
   int fidx[kPool];      // final node index of a pool entry
-  double prevkey[kMaxBudget];  // depth d-1 survivors, in order
-  int prevpid[kMaxBudget];
-  double lkey[kMaxBudget];     // best candidates of depth d, in order
-  int ljr[kMaxBudget];         // (parent position << 4) | rank
-  double gkey[2][kMaxBudget];  // global order so far (double-buffered)
+  double lkey[2][kMaxBudget];  // candidates of a depth in pop order (best first)
+  int ljr[2][kMaxBudget];      // (parent position << 4) | rank
+  double gkey[2][kMaxBudget];  // global order so far
   int gpid[2][kMaxBudget];
+  int n_kept[3], n_surv[3];    // per depth, d % 3 (reset two depths after their last read)
 };
 
 size_t expand_dyn_smem() { return sizeof(SelectSmem); }
@@ -319,7 +319,23 @@ __device__ void expand_sequential(ExpandSmem& s, int lane, int max_depth, int to
   }
 }
 
-__global__ void __launch_bounds__(kThreads)
+// First position in [0, n) (n <= kMaxBudget) at which pred fails, for a pred that holds on a prefix;
+// R searches run interleaved (independent load chains), branch-free.
+template <int R, class Pred>
+__device__ __forceinline__ void prefix_lengths(int n, int (&cnt)[R], Pred pred) {
+#pragma unroll
+  for (int i = 0; i < R; ++i) cnt[i] = 0;
+  for (int step = n > 0 ? (1 << (31 - __clz(n))) : 0; step > 0; step >>= 1) {
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int t = cnt[i] + step;
+      if (t <= n && pred(i, t - 1)) cnt[i] = t;
+    }
+  }
+}
+
+template <int K>
+__global__ void __launch_bounds__(kExpandThreads)
     expand_kernel(const RowPartial* __restrict__ part, int nchunks, const int32_t* __restrict__ root_tokens,
                   int max_depth, int topk, int budget, int32_t* __restrict__ parent, int32_t* __restrict__ token,
                   float* __restrict__ score, int32_t* __restrict__ depth_out) {
@@ -328,30 +344,30 @@ __global__ void __launch_bounds__(kThreads)
   SelectSmem& q = *reinterpret_cast<SelectSmem*>(dyn);
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // ---- 1. per-depth lse (float64) and top-k
-  for (int d = 1 + warp; d <= max_depth; d += kThreads / 32) {
+  // ---- 1. per-depth lse (float64) and top-k: one warp per depth, one lane per chunk partial
+  for (int d = 1 + warp; d <= max_depth; d += kExpandThreads / 32) {
     const RowPartial* rp = part + (static_cast<long long>(b) * max_depth + (d - 1)) * nchunks;
     float m = -INFINITY;
     for (int c = lane; c < nchunks; c += 32) m = fmaxf(m, rp[c].m);
     m = warp_max_f(m);
     const double md = static_cast<double>(m);
     double sum = 0.0;
-    Cand t[kMaxTopk];
+    Cand t[K];
 #pragma unroll
-    for (int i = 0; i < kMaxTopk; ++i) t[i] = Cand{-INFINITY, INT_MAX};
+    for (int i = 0; i < K; ++i) t[i] = Cand{-INFINITY, INT_MAX};
     for (int c = lane; c < nchunks; c += 32) {
       sum += rp[c].sum * exp_nonpos_f64(static_cast<double>(rp[c].m) - md);
-      Cand u[kMaxTopk];
+      Cand u[K];
 #pragma unroll
-      for (int i = 0; i < kMaxTopk; ++i) u[i] = Cand{rp[c].val[i], rp[c].id[i]};
-      merge8(t, u);
+      for (int i = 0; i < K; ++i) u[i] = Cand{rp[c].val[i], rp[c].id[i]};
+      merge_k<K>(t, u);
     }
     sum = warp_sum_d(sum);
-    warp_merge8(t, 32);
+    warp_merge_k<K>(t, 32);
     if (lane == 0) {
       const double lse = md + log(sum);
 #pragma unroll
-      for (int r = 0; r < kMaxTopk; ++r) {
+      for (int r = 0; r < K; ++r) {
         s.lp[d][r] = static_cast<double>(t[r].v) - lse;
         s.tok[d][r] = t[r].id;
       }
@@ -366,114 +382,113 @@ __global__ void __launch_bounds__(kThreads)
     tok_o[0] = root_tokens[b];
     sc_o[0] = 0.f;
     if (dep_o) dep_o[0] = 0;
+    q.lkey[0][0] = 0.0;  // "depth 0": the root
+    q.n_kept[1] = 0;
+    q.n_surv[1] = 0;
   }
   const int T = budget - 1;
   if (T == 0) return;
-  // ---- 2. level-parallel selection of the T best nodes in pop order
-  if (tid == 0) {
-    q.prevkey[0] = 0.0;
-    q.prevpid[0] = -1;
-  }
   __syncthreads();
-  int n_prev = 1, g = 0, cur = 0, pool_base = 0;
+  // ---- 2. level-parallel selection of the T best nodes in pop order.  Depth d reads the survivors of
+  // depth d - 1 (list buffer (d - 1) & 1, a prefix of n_prev entries) and writes buffer d & 1.
+  int n_prev = 1, g = 0, cur = 0, pool_base = 0, prev_base = -1;
   bool overflow = false;
   for (int d = 1; d <= max_depth; ++d) {
     if (n_prev == 0) break;
+    const int pb = (d - 1) & 1, cb = d & 1;
+    const double* prevkey = q.lkey[pb];
     const bool full = (g == T);
     const double thr = full ? q.gkey[cur][T - 1] : 0.0;
-    if (full && !(q.prevkey[0] + s.lp[d][0] > thr)) break;  // no depth-d node can enter
-    if (tid == 0) {
-      s.n_kept = 0;
-      s.n_surv = 0;
+    if (full && !(prevkey[0] + s.lp[d][0] > thr)) break;  // no depth-d node can enter
+    const int ci = d % 3;
+    if (tid == 0) {  // counters of depth d + 1, last read at depth d - 2 (before this depth's barriers)
+      q.n_kept[(d + 1) % 3] = 0;
+      q.n_surv[(d + 1) % 3] = 0;
     }
-    __syncthreads();
+    // (a) rank every candidate (j, r) = (parent at position j, rank r) among depth d's candidates.
+    // Order: key desc, then parent position, then rank.  Candidates of rank r2 that precede it form a
+    // prefix of the parents list (keys are non-increasing along it).
     const double* lpd = s.lp[d];
     const int nc = n_prev * topk;
-    for (int idx = tid; idx < nc; idx += kThreads) {
+    int kept = 0;
+    for (int idx = tid; idx < nc; idx += kExpandThreads) {
       const int j = idx / topk;
       const int r = idx - j * topk;
-      const double kc = q.prevkey[j] + lpd[r];
+      const double kc = prevkey[j] + lpd[r];
       if (full && !(kc > thr)) continue;  // cannot beat the current T-th node (ties go to shallower)
-      atomicAdd(&s.n_kept, 1);
-      int pos = j;  // candidates (j' < j, r) of its own list come first
-      for (int r2 = 0; r2 < topk; ++r2) {
-        if (r2 == r) continue;
-        int lo, hi;
-        if (r2 < r) { lo = j + 1; hi = n_prev; pos += 0; } else { lo = 0; hi = j; }
-        const double l2 = lpd[r2];
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          const double a = q.prevkey[mid] + l2;
-          const bool prec = a > kc || (a == kc && (mid < j || (mid == j && r2 < r)));
-          if (prec) lo = mid + 1; else hi = mid;
-        }
-        pos += lo;
-      }
+      ++kept;
+      int cnt[K];
+      prefix_lengths<K>(n_prev, cnt, [&](int r2, int jj) {
+        const double a = prevkey[jj] + lpd[r2];
+        return a > kc || (a == kc && (jj < j || (jj == j && r2 < r)));
+      });
+      int pos = 0;
+#pragma unroll
+      for (int r2 = 0; r2 < K; ++r2)
+        if (r2 < topk) pos += (r2 == r) ? j : cnt[r2];
       if (pos < T) {
-        q.lkey[pos] = kc;
-        q.ljr[pos] = (j << 4) | r;
+        q.lkey[cb][pos] = kc;
+        q.ljr[cb][pos] = (j << 4) | r;
       }
     }
+    kept = __reduce_add_sync(0xffffffffu, kept);
+    if (lane == 0 && kept) atomicAdd(&q.n_kept[ci], kept);
     __syncthreads();
-    const int n_d = min(s.n_kept, T);
-    // merge the global order (g entries) with the depth-d list (n_d entries); equal keys: shallower first
-    for (int i = tid; i < g; i += kThreads) {
+    const int n_d = min(q.n_kept[ci], T);
+    const double* lk = q.lkey[cb];
+    // (b) merge the global order (g entries) with the depth-d list (n_d entries), keeping T; equal keys:
+    // the global (shallower) entry first
+    for (int i = tid; i < g; i += kExpandThreads) {
       const double gk = q.gkey[cur][i];
-      int lo = 0, hi = n_d;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (q.lkey[mid] > gk) lo = mid + 1; else hi = mid;
-      }
-      const int pos = i + lo;
+      int c1[1];
+      prefix_lengths<1>(n_d, c1, [&](int, int jj) { return lk[jj] > gk; });
+      const int pos = i + c1[0];
       if (pos < T) {
         q.gkey[cur ^ 1][pos] = gk;
         q.gpid[cur ^ 1][pos] = q.gpid[cur][i];
       }
     }
-    for (int j = tid; j < n_d; j += kThreads) {
-      const double lk = q.lkey[j];
-      int lo = 0, hi = g;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (q.gkey[cur][mid] >= lk) lo = mid + 1; else hi = mid;
-      }
-      const int pos = j + lo;
+    int surv = 0;
+    for (int j = tid; j < n_d; j += kExpandThreads) {
+      const double k = lk[j];
+      int c1[1];
+      prefix_lengths<1>(g, c1, [&](int, int ii) { return q.gkey[cur][ii] >= k; });
+      const int pos = j + c1[0];
       if (pos < T) {
         const int pid = pool_base + j;
-        atomicMax(&s.n_surv, j + 1);
+        surv = j + 1;
         if (pid < kPool) {
-          const int jr = q.ljr[j];
-          q.pool_key[pid] = lk;
-          q.pool_par[pid] = q.prevpid[jr >> 4];
+          const int jr = q.ljr[cb][j];
+          q.pool_key[pid] = k;
+          q.pool_par[pid] = (d == 1) ? -1 : prev_base + (jr >> 4);
           q.pool_dr[pid] = (d << 8) | (jr & 15);
         }
-        q.gkey[cur ^ 1][pos] = lk;
+        q.gkey[cur ^ 1][pos] = k;
         q.gpid[cur ^ 1][pos] = pid;
       }
     }
+    surv = __reduce_max_sync(0xffffffffu, surv);
+    if (lane == 0 && surv) atomicMax(&q.n_surv[ci], surv);
     __syncthreads();
-    const int n_surv = s.n_surv;
+    const int n_surv = q.n_surv[ci];
     if (pool_base + n_surv > kPool) {
       overflow = true;
       break;
     }
-    for (int j = tid; j < n_surv; j += kThreads) {
-      q.prevkey[j] = q.lkey[j];
-      q.prevpid[j] = pool_base + j;
-    }
+    prev_base = pool_base;
     pool_base += n_surv;
     n_prev = n_surv;
     g = min(g + n_d, T);
     cur ^= 1;
-    __syncthreads();
   }
   if (overflow || g < T) {
+    __syncthreads();
     if (warp == 0) expand_sequential(s, lane, max_depth, topk, budget, par_o, tok_o, sc_o, dep_o);
     return;
   }
-  for (int i = tid; i < T; i += kThreads) q.fidx[q.gpid[cur][i]] = i + 1;
+  for (int i = tid; i < T; i += kExpandThreads) q.fidx[q.gpid[cur][i]] = i + 1;
   __syncthreads();
-  for (int i = tid; i < T; i += kThreads) {
+  for (int i = tid; i < T; i += kExpandThreads) {
     const int pid = q.gpid[cur][i];
     const int dr = q.pool_dr[pid];
     const int d = dr >> 8, r = dr & 255;
@@ -515,12 +530,29 @@ cudaError_t launch_build_tree(const float* logits, const int32_t* root_tokens, i
   if (dev < 0) return cudaErrorInvalidDevice;
   const size_t dyn = build::expand_dyn_smem();
   if (!attr_set[dev].load(std::memory_order_acquire)) {
-    e = cudaFuncSetAttribute(build::expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn));
-    if (e != cudaSuccess) return e;
+    const void* fns[4] = {reinterpret_cast<const void*>(build::expand_kernel<1>),
+                          reinterpret_cast<const void*>(build::expand_kernel<2>),
+                          reinterpret_cast<const void*>(build::expand_kernel<4>),
+                          reinterpret_cast<const void*>(build::expand_kernel<8>)};
+    for (const void* f : fns) {
+      e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn));
+      if (e != cudaSuccess) return e;
+    }
     attr_set[dev].store(true, std::memory_order_release);
   }
-  build::expand_kernel<<<batch, build::kThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth, topk,
-                                                                budget, parent, token, score, depth);
+  const dim3 g2(batch);
+  if (topk <= 1)
+    build::expand_kernel<1><<<g2, build::kExpandThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth,
+                                                                        topk, budget, parent, token, score, depth);
+  else if (topk <= 2)
+    build::expand_kernel<2><<<g2, build::kExpandThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth,
+                                                                        topk, budget, parent, token, score, depth);
+  else if (topk <= 4)
+    build::expand_kernel<4><<<g2, build::kExpandThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth,
+                                                                        topk, budget, parent, token, score, depth);
+  else
+    build::expand_kernel<8><<<g2, build::kExpandThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth,
+                                                                        topk, budget, parent, token, score, depth);
   return cudaGetLastError();
 }
 

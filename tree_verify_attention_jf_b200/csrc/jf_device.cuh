@@ -252,30 +252,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
   return r;
 }
 
-// 2^y for a pair of floats on the FMA pipe, for y <= 8.  y = n + f with n = round(y) (added to the
-// exponent field) and f in [-1/2, 1/2], where 2^f is a cubic fitted to minimise the relative error
-// (max 1.4e-4, far below the 2^-9 rounding of the bf16 result).  y < -125 (and -inf) gives 0.
-__device__ __forceinline__ void exp2_poly2(uint64_t y2, float& p0, float& p1) {
-  const uint64_t magic = f2_pack(12582912.f, 12582912.f);    // 1.5 * 2^23
-  const uint64_t nmagic = f2_pack(-12582912.f, -12582912.f);
-  const uint64_t m1 = f2_pack(-1.f, -1.f);
-  float y0, y1;
-  f2_unpack(y2, y0, y1);
-  const uint64_t yc = f2_pack(fmaxf(y0, -127.f), fmaxf(y1, -127.f));
-  const uint64_t t = f2_add(yc, magic);            // low mantissa bits of t hold round(y)
-  const uint64_t f = f2_fma(f2_add(t, nmagic), m1, yc);
-  uint64_t p = f2_fma(f2_pack(0x1.c66710p-5f, 0x1.c66710p-5f), f, f2_pack(0x1.f06bc0p-3f, 0x1.f06bc0p-3f));
-  p = f2_fma(p, f, f2_pack(0x1.62e9b8p-1f, 0x1.62e9b8p-1f));
-  p = f2_fma(p, f, f2_pack(0x1.fff81cp-1f, 0x1.fff81cp-1f));
-  float q0, q1, t0, t1;
-  f2_unpack(p, q0, q1);
-  f2_unpack(t, t0, t1);
-  const int n0 = __float_as_int(t0) - __float_as_int(12582912.f);
-  const int n1 = __float_as_int(t1) - __float_as_int(12582912.f);
-  p0 = y0 < -125.f ? 0.f : __int_as_float(__float_as_int(q0) + (n0 << 23));
-  p1 = y1 < -125.f ? 0.f : __int_as_float(__float_as_int(q1) + (n1 << 23));
-}
-
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

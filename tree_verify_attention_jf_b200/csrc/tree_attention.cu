@@ -44,10 +44,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmS = 0;    // S_i at column 128 * i
 constexpr uint32_t kTmO = 256;  // O_i at column 256 + 128 * i
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow up to 2^8 before O is rescaled
-// Pairs of P (bit i: columns 2i, 2i+1 of each 64-column half) whose 2^y is evaluated on the FMA pipe
-// by a polynomial instead of by MUFU ex2: the two softmax warpgroups share each SM's 16 ex2 per
-// clock, and moving part of the work to the otherwise idle FMA pipe shortens the exp phase.
-constexpr uint32_t kPolyPairs = 0x00000000u;
 
 struct __align__(1024) Smem {
   uint8_t q[kAttnQTiles][kTileBytes];
@@ -503,34 +499,37 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
         meta_seen = true;
       }
       if (!warp_wait(&s.bar_sfull[qt], it & 1, abort)) return set_abort(s, p);
-      // S_qt(it) ready implies PV_qt(it-1) is complete (the tensor pipe runs in issue order); observing
-      // that phase keeps the pv-done barrier in step for the epilogue's wait.
-      if (it >= 1 && !warp_wait(&s.bar_pvdone[qt], (it - 1) & 1, abort)) return set_abort(s, p);
+      // S_qt(it) ready also means PV_qt(it-1) is complete: its commit tracks every earlier MMA.
       tc_fence_after();
-      // the whole 128-column row of S in registers: one TMEM round trip per tile
+      // The row of S in registers, in two halves: the max of the first half is taken while the
+      // second half is still on its way from TMEM.
       uint32_t sr[128];
       tmem_ld32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(lane_base + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      tmem_ld32(lane_base + s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       uint32_t vis[4];
 #pragma unroll
       for (int w = 0; w < 4; ++w)
         vis[w] = tree_tile ? vis_word(t * kBN + 32 * w, g.P, g.N, row_valid, anc) : 0xffffffffu;
       tmem_ld_wait();
-      if (tree_tile) {
-        // invisible keys become -inf: they drop out of the max and get P = 2^-inf = 0
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (!((vis[c >> 5] >> (c & 31)) & 1u)) sr[c] = 0xff800000u;
-      }
+      tmem_ld32(lane_base + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(lane_base + s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; c += 8) {
-        a0 = fmax3(a0, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
-        a1 = fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-        a2 = fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-        a3 = fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+      for (int hh = 0; hh < 2; ++hh) {
+        if (hh == 1) tmem_ld_wait();
+        if (tree_tile) {
+          // invisible keys become -inf: they drop out of the max and get P = 2^-inf = 0
+#pragma unroll
+          for (int c = 64 * hh; c < 64 * hh + 64; ++c)
+            if (!((vis[c >> 5] >> (c & 31)) & 1u)) sr[c] = 0xff800000u;
+        }
+#pragma unroll
+        for (int c = 64 * hh; c < 64 * hh + 64; c += 8) {
+          a0 = fmax3(a0, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
+          a1 = fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+          a2 = fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+          a3 = fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+        }
       }
       const float mraw = fmax3(a0, a1, fmaxf(a2, a3));
       const float mx = (mraw == -INFINITY) ? -INFINITY : mraw * sl2;
@@ -546,29 +545,24 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
       }
       const float negm = (m_use == -INFINITY) ? 0.f : -m_use;
       const uint64_t nm2 = f2_pack(negm, negm);
-      // P = 2^(s * scale - m), row sum in packed pairs, bf16 pairs of P written over S's first 64 columns
+      // P = 2^(s * scale - m), row sum in packed pairs, bf16 pairs of P written over S's first 64
+      // columns, a quarter (16 packed columns) at a time
       uint64_t acc0 = 0, acc1 = 0;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {  // two halves, so only 32 packed words are live at a time
-        uint32_t pk[32];
+      for (int h = 0; h < 4; ++h) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const int cc = 64 * h + c;
+        for (int c = 0; c < 32; c += 2) {
+          const int cc = 32 * h + c;
           const uint64_t y = f2_fma(f2_pack(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), sl2x2, nm2);
-          float p0, p1;
-          if ((kPolyPairs >> (c >> 1)) & 1u) {
-            exp2_poly2(y, p0, p1);
-          } else {
-            float y0, y1;
-            f2_unpack(y, y0, y1);
-            p0 = ex2_approx(y0);
-            p1 = ex2_approx(y1);
-          }
+          float y0, y1;
+          f2_unpack(y, y0, y1);
+          const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
           if ((c >> 1) & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
           else acc0 = f2_add(acc0, f2_pack(p0, p1));
           pk[c >> 1] = pack_bf16x2_alu(p0, p1);
         }
-        tmem_st32(lane_base + s_col + 32 * h, pk);
+        tmem_st16(lane_base + s_col + 16 * h, pk);
       }
       {
         float u0, u1, v0, v1;
@@ -742,91 +736,129 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------------
-// Combine kernel: merges the partials of every unit that was cut between CTAs.  Block (c0, q, rb)
-// handles rows [32 rb, 32 rb + 32) of M tile q of the unit whose first CTA is c0; each of its 256
-// threads owns one row and four 4-column groups and loads the unit's segments four at a time (a unit
-// cut into at most four pieces is merged in one memory round trip).
+// Combine kernel: merges the partials of every unit that was cut between CTAs.  A fixed grid (two
+// blocks per SM) first compacts the split units out of the descriptor table (one slot per attention
+// CTA) and then takes work items (split unit, M tile, 32-row block) in a grid-stride loop.  A thread
+// owns one row and four 4-column groups and merges the unit's segments in a single pass with a
+// running max, loading kSegBatch segments at a time (one memory round trip per batch).
 // Launched right after the attention kernel (programmatic dependent launch), it waits for the
 // attention grid before reading.
 // ------------------------------------------------------------------------------------------------
+constexpr int kCombineThreads = 256;
 constexpr int kCombineRows = 32;
 constexpr int kCombineQuads = 4;  // 4-column groups per thread
 constexpr int kSegBatch = 4;      // segments whose partials are loaded in one batch
+constexpr int kItemsPerUnit = kAttnQTiles * (kBM / kCombineRows);
 
-__global__ void __launch_bounds__(256, 2) combine_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnParams p, int ncta) {
+  static_assert(kMaxGrid <= kCombineThreads, "one descriptor slot per thread");
+  __shared__ int4 s_desc[kMaxGrid];
+  __shared__ int s_c0[kMaxGrid];
+  __shared__ int s_wcount[kCombineThreads / 32];
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the attention grid has completed
-  const int c0 = blockIdx.x;
-  const int qt = blockIdx.y;
-  const int rb = blockIdx.z;
-  const int4 d = __ldcg(&p.units[c0]);
-  const int c1 = d.x;
-  if (c1 <= c0) return;  // no split unit starts at this CTA
-  const int rl = threadIdx.x & (kCombineRows - 1);
-  const int q0 = (threadIdx.x >> 5) * kCombineQuads;  // first 4-column group of this thread
-  const int r = rb * kCombineRows + rl;               // row of the M tile
-  const int nodes_per_tile = kBM / p.group;
-  const int node = qt * nodes_per_tile + r / p.group;
-  if (node >= d.z) return;
-  const long long grow = static_cast<long long>(d.y + node) * p.hq + d.w * p.group + (r % p.group);
-  float M = -INFINITY;
-  bool ok = true;
-  for (int cb = c0; cb <= c1; cb += kSegBatch) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // Compact the split units in CTA order (the same list in every block, so that work item i means
+  // the same unit everywhere): thread c reads slot c.
+  int4 dc = make_int4(0, 0, 0, 0);
+  if (tid < ncta) dc = __ldcg(&p.units[tid]);
+  const bool split_here = tid < ncta && dc.x > tid;  // a split unit starts at CTA tid and ends at dc.x
+  const uint32_t bal = __ballot_sync(0xffffffffu, split_here);
+  if (lane == 0) s_wcount[warp] = __popc(bal);
+  __syncthreads();
+  int base = 0, total = 0;
 #pragma unroll
-    for (int u = 0; u < kSegBatch; ++u) {
-      const int c = cb + u;
-      if (c <= c1) {
-        const int sl = slot_of(c, c0) * kAttnQTiles + qt;
-        M = fmaxf(M, __ldcg(&p.part_ml[static_cast<long long>(sl) * kBM + r]).x);
-        ok = ok && __ldcg(&p.part_ok[static_cast<long long>(sl) * kBM + r]) != 0;
-      }
-    }
+  for (int w = 0; w < kCombineThreads / 32; ++w) {
+    base += (w < warp) ? s_wcount[w] : 0;
+    total += s_wcount[w];
   }
-  float L = 0.f;
-  float4 acc[kCombineQuads];
+  if (split_here) {
+    const int k = base + __popc(bal & ((1u << lane) - 1u));
+    s_desc[k] = dc;
+    s_c0[k] = tid;
+  }
+  __syncthreads();
+  const int s_n = total;
+  const int n_items = s_n * kItemsPerUnit;
+  const int rl = lane;
+  const int q0 = warp * kCombineQuads;  // first 4-column group of this thread
+  const int nodes_per_tile = kBM / p.group;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int u = item / kItemsPerUnit;
+    const int qt = (item / (kBM / kCombineRows)) % kAttnQTiles;
+    const int rb = item % (kBM / kCombineRows);
+    const int4 d = s_desc[u];
+    const int c0 = s_c0[u], c1 = d.x;
+    const int r = rb * kCombineRows + rl;  // row of the M tile
+    const int node = qt * nodes_per_tile + r / p.group;
+    if (node >= d.z) continue;
+    const long long grow = static_cast<long long>(d.y + node) * p.hq + d.w * p.group + (r % p.group);
+    float M = -INFINITY, L = 0.f;
+    bool ok = true;
+    float4 acc[kCombineQuads];
 #pragma unroll
-  for (int q = 0; q < kCombineQuads; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int cb = c0; cb <= c1; cb += kSegBatch) {
-    float2 ml[kSegBatch];
-    float4 v[kSegBatch][kCombineQuads];
+    for (int q = 0; q < kCombineQuads; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int cb = c0; cb <= c1; cb += kSegBatch) {
+      float2 ml[kSegBatch];
+      int okv[kSegBatch];
+      float4 v[kSegBatch][kCombineQuads];
 #pragma unroll
-    for (int u = 0; u < kSegBatch; ++u) {
-      const int c = cb + u;
-      const int sl = slot_of(c, c0) * kAttnQTiles + qt;
-      const bool have = c <= c1;
-      ml[u] = have ? __ldcg(&p.part_ml[static_cast<long long>(sl) * kBM + r]) : make_float2(-INFINITY, 0.f);
+      for (int j = 0; j < kSegBatch; ++j) {
+        const int c = cb + j;
+        const bool have = c <= c1;
+        const int sl = slot_of(c, c0) * kAttnQTiles + qt;
+        ml[j] = have ? __ldcg(&p.part_ml[static_cast<long long>(sl) * kBM + r]) : make_float2(-INFINITY, 0.f);
+        okv[j] = have ? __ldcg(&p.part_ok[static_cast<long long>(sl) * kBM + r]) : 1;
 #pragma unroll
-      for (int q = 0; q < kCombineQuads; ++q)
-        v[u][q] = have ? __ldcg(part_ptr(p, sl, q0 + q, r)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+        for (int q = 0; q < kCombineQuads; ++q)
+          v[j][q] = have ? __ldcg(part_ptr(p, sl, q0 + q, r)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float Mb = M;
 #pragma unroll
-    for (int u = 0; u < kSegBatch; ++u) {
-      if (ml[u].x == -INFINITY) continue;
-      const float w = ex2_approx(ml[u].x - M);
-      L = fmaf(w, ml[u].y, L);
+      for (int j = 0; j < kSegBatch; ++j) {
+        Mb = fmaxf(Mb, ml[j].x);
+        ok = ok && okv[j] != 0;
+      }
+      if (Mb == -INFINITY) continue;  // nothing visible so far
+      const float a = ex2_approx(M - Mb);  // 0 while M is still -inf
+      L *= a;
 #pragma unroll
       for (int q = 0; q < kCombineQuads; ++q) {
-        acc[q].x = fmaf(w, v[u][q].x, acc[q].x);
-        acc[q].y = fmaf(w, v[u][q].y, acc[q].y);
-        acc[q].z = fmaf(w, v[u][q].z, acc[q].z);
-        acc[q].w = fmaf(w, v[u][q].w, acc[q].w);
+        acc[q].x *= a;
+        acc[q].y *= a;
+        acc[q].z *= a;
+        acc[q].w *= a;
       }
+#pragma unroll
+      for (int j = 0; j < kSegBatch; ++j) {
+        if (ml[j].x == -INFINITY) continue;
+        const float w = ex2_approx(ml[j].x - Mb);
+        L = fmaf(w, ml[j].y, L);
+#pragma unroll
+        for (int q = 0; q < kCombineQuads; ++q) {
+          acc[q].x = fmaf(w, v[j][q].x, acc[q].x);
+          acc[q].y = fmaf(w, v[j][q].y, acc[q].y);
+          acc[q].z = fmaf(w, v[j][q].z, acc[q].z);
+          acc[q].w = fmaf(w, v[j][q].w, acc[q].w);
+        }
+      }
+      M = Mb;
     }
+    if (!ok) continue;
+    const float inv = 1.f / L;
+    uint4 o[2];
+    o[0].x = pack_bf16x2(acc[0].x * inv, acc[0].y * inv);
+    o[0].y = pack_bf16x2(acc[0].z * inv, acc[0].w * inv);
+    o[0].z = pack_bf16x2(acc[1].x * inv, acc[1].y * inv);
+    o[0].w = pack_bf16x2(acc[1].z * inv, acc[1].w * inv);
+    o[1].x = pack_bf16x2(acc[2].x * inv, acc[2].y * inv);
+    o[1].y = pack_bf16x2(acc[2].z * inv, acc[2].w * inv);
+    o[1].z = pack_bf16x2(acc[3].x * inv, acc[3].y * inv);
+    o[1].w = pack_bf16x2(acc[3].z * inv, acc[3].w * inv);
+    uint4* dst = reinterpret_cast<uint4*>(p.out + grow * 128 + q0 * 4);
+    dst[0] = o[0];
+    dst[1] = o[1];
+    if (q0 == 0 && p.lse != nullptr) p.lse[grow] = (M + __log2f(L)) * 0.69314718055994531f;
   }
-  if (!ok) return;
-  const float inv = 1.f / L;
-  uint4 o[2];
-  o[0].x = pack_bf16x2(acc[0].x * inv, acc[0].y * inv);
-  o[0].y = pack_bf16x2(acc[0].z * inv, acc[0].w * inv);
-  o[0].z = pack_bf16x2(acc[1].x * inv, acc[1].y * inv);
-  o[0].w = pack_bf16x2(acc[1].z * inv, acc[1].w * inv);
-  o[1].x = pack_bf16x2(acc[2].x * inv, acc[2].y * inv);
-  o[1].y = pack_bf16x2(acc[2].z * inv, acc[2].w * inv);
-  o[1].z = pack_bf16x2(acc[3].x * inv, acc[3].y * inv);
-  o[1].w = pack_bf16x2(acc[3].z * inv, acc[3].w * inv);
-  uint4* dst = reinterpret_cast<uint4*>(p.out + grow * 128 + q0 * 4);
-  dst[0] = o[0];
-  dst[1] = o[1];
-  if (q0 == 0 && p.lse != nullptr) p.lse[grow] = (M + __log2f(L)) * 0.69314718055994531f;
 }
 
 }  // namespace attn
@@ -854,12 +886,12 @@ cudaError_t launch_tree_attention(const CUtensorMap& tm_q, const CUtensorMap& tm
   attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr.val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, kAttnQTiles, kAttnRows / attn::kCombineRows);
-  cfg.blockDim = dim3(256);
+  cfg.gridDim = dim3(2 * grid);
+  cfg.blockDim = dim3(attn::kCombineThreads);
   cfg.stream = stream;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn::combine_kernel, p);
+  return cudaLaunchKernelEx(&cfg, attn::combine_kernel, p, grid);
 }
 
 }  // namespace jf
