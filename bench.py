@@ -40,6 +40,11 @@ HEAD_DIM = 128
 PAGE = 16
 L2_FLUSH_BYTES = 256 << 20
 LAUNCHES_PER_STEP = 5
+# DRAM traffic of one tree_attention_kernel launch on the default workload (dram__bytes_read.sum +
+# dram__bytes_write.sum from the capture summarised in profiles/tree_attention_kernel_qwen3_8b.md), valid
+# only for the kernel source it was taken on: the roofline reports null once that source has changed.
+ATTN_TRAFFIC = {"qwen3_8b": {"bytes": 20.014080e6 + 0.014848e6,
+                             "source_sha256": "3245e97978596ad4eab819431ec28bc46815ea6653a257a672b238bf5c828868"}}
 
 
 def peaks():
@@ -67,6 +72,19 @@ def make_inputs(cfg, seed):
     kv_shape = (num_pages, PAGE, cfg["hkv"], HEAD_DIM)
     return dict(draft=x, roots=roots, q=q, kv_shape=kv_shape, block_table=bt, prefix=np.array(prefix, np.int32),
                 offsets=(np.arange(B + 1) * N).astype(np.int32))
+
+
+def attention_traffic(workload):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary, if the kernel source is
+    still the one that was profiled; else None."""
+    import hashlib
+    rec = ATTN_TRAFFIC.get(workload)
+    if rec is None:
+        return None
+    src = os.path.join(ROOT, "tree_verify_attention_jf_b200", "csrc", "tree_attention.cu")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    return rec["bytes"] if digest == rec["source_sha256"] else None
 
 
 def rank_seed(rank):
@@ -386,8 +404,9 @@ def main():
         "metric": metric, "value": job_nodes_per_sec(B, N, world, step_ms), "unit": "nodes/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)", "config": config,
-        "roofline": {"kernel": "jf::attn::tree_attention_kernel", "bound": "tensor", "achieved": tflops,
-                     "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops / pk["bf16"], "traffic": None,
+        "roofline": {"kernel": "jf_tree_attention (tree_attention_kernel + combine_kernel)", "bound": "tensor",
+                     "achieved": tflops, "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops / pk["bf16"],
+                     "traffic": attention_traffic(args.workload),
                      "peak_source": pk["src"] + " bf16 burst",
                      "hbm_achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm"],
                      "algorithmic_flops": flops, "algorithmic_bytes": kv_bytes + qo_bytes + meta_bytes},

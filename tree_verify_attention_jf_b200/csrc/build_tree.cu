@@ -191,7 +191,10 @@ __global__ void __launch_bounds__(kThreads)
 // ------------------------------------------------------------------------------------------------
 // Kernel 2: merge + best-first expansion.  grid = batch, block = 256
 // ------------------------------------------------------------------------------------------------
+// Order-preserving map of a (non-NaN) double to an unsigned integer: a < b as doubles iff
+// ord_key(a) < ord_key(b).  -0 is taken as +0 so that equal doubles give equal keys.
 __device__ __forceinline__ unsigned long long ord_key(double k) {
+  if (k == 0.0) k = 0.0;
   const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(k));
   return (bits >> 63) ? ~bits : (bits | 0x8000000000000000ull);
 }
@@ -211,18 +214,22 @@ struct ExpandSmem {
 // Level-parallel selection state (dynamic shared memory).  Nodes are kept in a pool in creation
 // order; lists hold pool ids.  The depth lists are double-buffered: the survivors of depth d (a prefix
 // of its list) are the parents of depth d + 1.
-constexpr int kPool = 4096;
+constexpr int kPool = 2048;
 constexpr int kExpandThreads = 512;
 struct SelectSmem {
   double pool_key[kPool];
   int pool_par[kPool];  // parent's pool id, -1 = the root
   int pool_dr[kPool];   // (depth << 8) | rank
   int fidx[kPool];      // final node index of a pool entry
-  double lkey[2][kMaxBudget];  // candidates of a depth in pop order (best first)
-  int ljr[2][kMaxBudget];      // (parent position << 4) | rank
-  double gkey[2][kMaxBudget];  // global order so far
+  // All ordering decisions compare order-preserving integer images of the float64 keys: integer
+  // compares have a short latency, while a search runs a long chain of dependent compares.
+  unsigned long long cord[kMaxTopk][kMaxBudget];  // key of candidate (parent position j, rank r) at [r][j]
+  double lkey[2][kMaxBudget];              // candidates of a depth in pop order (best first)
+  unsigned long long lord[2][kMaxBudget];  // their integer keys
+  int ljr[2][kMaxBudget];                  // (parent position << 4) | rank
+  unsigned long long gord[2][kMaxBudget];  // global order so far (integer keys)
   int gpid[2][kMaxBudget];
-  int n_kept[3], n_surv[3];    // per depth, d % 3 (reset two depths after their last read)
+  int n_kept[3], n_surv[3];  // per depth, d % 3 (reset two depths after their last read)
 };
 
 size_t expand_dyn_smem() { return sizeof(SelectSmem); }
@@ -397,29 +404,36 @@ __global__ void __launch_bounds__(kExpandThreads)
     if (n_prev == 0) break;
     const int pb = (d - 1) & 1, cb = d & 1;
     const double* prevkey = q.lkey[pb];
+    const double* lpd = s.lp[d];
     const bool full = (g == T);
-    const double thr = full ? q.gkey[cur][T - 1] : 0.0;
-    if (full && !(prevkey[0] + s.lp[d][0] > thr)) break;  // no depth-d node can enter
+    const unsigned long long thr = full ? q.gord[cur][T - 1] : 0ull;
+    if (full && !(ord_key(prevkey[0] + lpd[0]) > thr)) break;  // no depth-d node can enter
     const int ci = d % 3;
     if (tid == 0) {  // counters of depth d + 1, last read at depth d - 2 (before this depth's barriers)
       q.n_kept[(d + 1) % 3] = 0;
       q.n_surv[(d + 1) % 3] = 0;
     }
-    // (a) rank every candidate (j, r) = (parent at position j, rank r) among depth d's candidates.
-    // Order: key desc, then parent position, then rank.  Candidates of rank r2 that precede it form a
-    // prefix of the parents list (keys are non-increasing along it).
-    const double* lpd = s.lp[d];
+    // (a) the float64 key of every candidate (j, r) = (parent at position j, rank r), as an integer key
     const int nc = n_prev * topk;
+    for (int idx = tid; idx < nc; idx += kExpandThreads) {
+      const int j = idx / topk;
+      const int r = idx - j * topk;
+      q.cord[r][j] = ord_key(prevkey[j] + lpd[r]);
+    }
+    __syncthreads();
+    // (b) rank every candidate among depth d's candidates.  Order: key desc, then parent position,
+    // then rank.  Candidates of rank r2 that precede it form a prefix of the parents list (keys are
+    // non-increasing along it).
     int kept = 0;
     for (int idx = tid; idx < nc; idx += kExpandThreads) {
       const int j = idx / topk;
       const int r = idx - j * topk;
-      const double kc = prevkey[j] + lpd[r];
+      const unsigned long long kc = q.cord[r][j];
       if (full && !(kc > thr)) continue;  // cannot beat the current T-th node (ties go to shallower)
       ++kept;
       int cnt[K];
       prefix_lengths<K>(n_prev, cnt, [&](int r2, int jj) {
-        const double a = prevkey[jj] + lpd[r2];
+        const unsigned long long a = q.cord[r2][jj];
         return a > kc || (a == kc && (jj < j || (jj == j && r2 < r)));
       });
       int pos = 0;
@@ -427,7 +441,8 @@ __global__ void __launch_bounds__(kExpandThreads)
       for (int r2 = 0; r2 < K; ++r2)
         if (r2 < topk) pos += (r2 == r) ? j : cnt[r2];
       if (pos < T) {
-        q.lkey[cb][pos] = kc;
+        q.lkey[cb][pos] = prevkey[j] + lpd[r];
+        q.lord[cb][pos] = kc;
         q.ljr[cb][pos] = (j << 4) | r;
       }
     }
@@ -435,35 +450,35 @@ __global__ void __launch_bounds__(kExpandThreads)
     if (lane == 0 && kept) atomicAdd(&q.n_kept[ci], kept);
     __syncthreads();
     const int n_d = min(q.n_kept[ci], T);
-    const double* lk = q.lkey[cb];
-    // (b) merge the global order (g entries) with the depth-d list (n_d entries), keeping T; equal keys:
+    const unsigned long long* lo = q.lord[cb];
+    // (c) merge the global order (g entries) with the depth-d list (n_d entries), keeping T; equal keys:
     // the global (shallower) entry first
     for (int i = tid; i < g; i += kExpandThreads) {
-      const double gk = q.gkey[cur][i];
+      const unsigned long long gk = q.gord[cur][i];
       int c1[1];
-      prefix_lengths<1>(n_d, c1, [&](int, int jj) { return lk[jj] > gk; });
+      prefix_lengths<1>(n_d, c1, [&](int, int jj) { return lo[jj] > gk; });
       const int pos = i + c1[0];
       if (pos < T) {
-        q.gkey[cur ^ 1][pos] = gk;
+        q.gord[cur ^ 1][pos] = gk;
         q.gpid[cur ^ 1][pos] = q.gpid[cur][i];
       }
     }
     int surv = 0;
     for (int j = tid; j < n_d; j += kExpandThreads) {
-      const double k = lk[j];
+      const unsigned long long k = lo[j];
       int c1[1];
-      prefix_lengths<1>(g, c1, [&](int, int ii) { return q.gkey[cur][ii] >= k; });
+      prefix_lengths<1>(g, c1, [&](int, int ii) { return q.gord[cur][ii] >= k; });
       const int pos = j + c1[0];
       if (pos < T) {
         const int pid = pool_base + j;
         surv = j + 1;
         if (pid < kPool) {
           const int jr = q.ljr[cb][j];
-          q.pool_key[pid] = k;
+          q.pool_key[pid] = q.lkey[cb][j];
           q.pool_par[pid] = (d == 1) ? -1 : prev_base + (jr >> 4);
           q.pool_dr[pid] = (d << 8) | (jr & 15);
         }
-        q.gkey[cur ^ 1][pos] = k;
+        q.gord[cur ^ 1][pos] = k;
         q.gpid[cur ^ 1][pos] = pid;
       }
     }

@@ -5,7 +5,9 @@
 // is split into a 32-bit head (so n * head is exact) and a tail; then e^r by its Taylor series
 // through r^13 (truncation below 5e-18 relative for |r| <= 0.3466), evaluated in Horner form with
 // fused multiply-adds; finally the exponent field is built from n.  Arguments below -708 return 0
-// (their terms are below 1e-307 next to a row maximum that contributes exactly 1).
+// (their terms are below 1e-307 next to a row maximum that contributes exactly 1).  n is rounded with
+// the 1.5 * 2^52 shift (the integer lands in the low mantissa bits), and the function has no
+// branches, so a thread's independent calls overlap.
 // Written from the mathematics above; the coefficients are 1/k!.
 #pragma once
 
@@ -26,9 +28,13 @@ JF_HD double exp_nonpos_f64(double x) {
   constexpr double kInvLn2 = 1.4426950408889634;
   constexpr double kLn2Hi = 0x1.62e42fee00000p-1;  // ln 2 with its low 21 mantissa bits cleared
   constexpr double kLn2Lo = 0x1.a39ef35793c76p-33;  // ln 2 - kLn2Hi
-  if (!(x >= -708.0)) return 0.0;  // also maps -inf / NaN to 0
-  const double n = rint(x * kInvLn2);
-  double r = fma(-n, kLn2Hi, x);
+  constexpr double kShift = 0x1.8p52;  // x / ln2 + kShift rounds x / ln2 to an integer in the low bits
+  // Branch-free: out-of-range arguments (below -708, -inf, NaN) are computed as 0 and replaced at the end.
+  const bool in_range = x >= -708.0;
+  const double xc = in_range ? x : 0.0;
+  const double t = fma(xc, kInvLn2, kShift);
+  const double n = t - kShift;  // rint(x / ln2), exact
+  double r = fma(-n, kLn2Hi, xc);
   r = fma(-n, kLn2Lo, r);
   double p = 1.0 / 6227020800.0;        // 1/13!
   p = fma(p, r, 1.0 / 479001600.0);     // 1/12!
@@ -44,15 +50,22 @@ JF_HD double exp_nonpos_f64(double x) {
   p = fma(p, r, 0.5);                   // 1/2!
   p = fma(p, r, 1.0);
   p = fma(p, r, 1.0);
-  // n in [-1022, 0]: 2^n is a normal double
-  const int64_t bits = static_cast<int64_t>(static_cast<int>(n) + 1023) << 52;
+  // n in [-1022, 0] sits in the low 32 bits of t; 2^n is a normal double
+  int64_t tb;
+#if defined(__CUDA_ARCH__)
+  tb = __double_as_longlong(t);
+#else
+  std::memcpy(&tb, &t, sizeof(tb));
+#endif
+  const int ni = static_cast<int>(static_cast<uint32_t>(tb));
+  const int64_t bits = static_cast<int64_t>(ni + 1023) << 52;
   double scale;
 #if defined(__CUDA_ARCH__)
   scale = __longlong_as_double(bits);
 #else
   std::memcpy(&scale, &bits, sizeof(scale));
 #endif
-  return p * scale;
+  return in_range ? p * scale : 0.0;
 }
 
 }  // namespace jf
