@@ -1,5 +1,7 @@
 """The float64 exp used by the draft-logit row sums, checked on the host against math.exp (an
-independent libm) within 2 ulp over the argument range the kernel sees, including the cutoff."""
+independent libm) over the argument range the kernel sees, including the cutoff, and its table of
+2^(j/32) against exact decimal arithmetic.  The bound is 1e-14 relative: the row sums only need to keep
+the tree's float64 keys within far less than the 1e-9 decision margins the build tests guard."""
 import math
 import os
 import shutil
@@ -21,22 +23,36 @@ def exe(tmp_path_factory):
     return str(out)
 
 
-def run(exe, xs):
-    res = subprocess.run([exe], input="\n".join(repr(float(x)) for x in xs), capture_output=True, text=True,
-                         check=True)
+def run(exe, xs, args=()):
+    res = subprocess.run([exe, *args], input="\n".join(repr(float(x)) for x in xs), capture_output=True,
+                         text=True, check=True)
     return np.array([float(v) for v in res.stdout.split()])
 
 
-def test_within_two_ulp(exe):
+def test_within_1e14_relative(exe):
     rng = np.random.default_rng(0)
     xs = np.concatenate([-rng.exponential(5.0, 4000), -rng.uniform(0, 708, 4000), -rng.uniform(0, 1e-3, 500),
                          [0.0, -0.0, -1e-300, -0.34657359027997264, -0.3465735902799727, -707.9, -1.0, -2.0]])
     got = run(exe, xs)
     want = np.array([math.exp(x) for x in xs])
-    ulp = np.abs(got - want) / np.spacing(want)
-    assert ulp.max() <= 2.0, (ulp.max(), xs[ulp.argmax()])
+    rel = np.abs(got - want) / want
+    assert rel.max() <= 1e-14, (rel.max(), xs[rel.argmax()])
 
 
 def test_cutoff_and_specials(exe):
     got = run(exe, [-708.5, -1e6, float("-inf"), 0.0])
     assert got[0] == 0.0 and got[1] == 0.0 and got[2] == 0.0 and got[3] == 1.0
+
+
+def test_table_is_correctly_rounded(exe):
+    from decimal import Decimal, getcontext
+    getcontext().prec = 60
+    res = subprocess.run([exe, "table"], capture_output=True, text=True, check=True)
+    tab = [float.fromhex(v) for v in res.stdout.split()]
+    assert len(tab) == 32
+    for j, d in enumerate(tab):
+        exact = Decimal(2) ** (Decimal(j) / Decimal(32))
+        err = abs(Decimal(d) - exact)
+        # no neighbouring double is closer
+        assert err <= abs(Decimal(math.nextafter(d, 0.0)) - exact), j
+        assert err <= abs(Decimal(math.nextafter(d, 4.0)) - exact), j

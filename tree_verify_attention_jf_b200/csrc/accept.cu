@@ -56,6 +56,12 @@ __device__ __forceinline__ void prefetch_l2(const float* p, long long n) {
   }
 }
 
+// all lanes of the warp wait (bounded) for the phase of `bar` with the given parity
+__device__ __forceinline__ bool warp_all_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
 __device__ __forceinline__ void warp_best(float& v, int& id) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -66,6 +72,21 @@ __device__ __forceinline__ void warp_best(float& v, int& id) {
 }
 
 constexpr int kWarps = kThreads / 32;
+
+// address of the same shared-memory variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t cluster_addr(const void* local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+  return r;
+}
+
+// 8-byte store into another CTA's shared memory that completes 8 bytes of transaction on that CTA's
+// mbarrier (the receiver learns of the data by waiting on its own barrier)
+__device__ __forceinline__ void st_async_best(uint32_t remote, float v, int id, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(remote),
+               "r"(__float_as_uint(v)), "r"(id), "r"(remote_bar)
+               : "memory");
+}
 
 __global__ void __launch_bounds__(kThreads)
     accept_kernel(const int32_t* __restrict__ token, const int32_t* __restrict__ parent,
@@ -78,9 +99,11 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ int s_off[kMaxAcceptNodes + 1];  // children of node n: s_kid[s_off[n] .. s_off[n + 1])
   __shared__ int s_kid[kMaxAcceptNodes];
   __shared__ int s_path[kMaxAcceptNodes + 1];
-  __shared__ Best s_part[kWarps];  // this step's per-warp partial argmax
-  __shared__ Best s_slot[2];       // this CTA's partial argmax, by step parity (read by the whole cluster)
-  __shared__ int2 s_dec[2];        // (argmax, next node) of the step, by step parity
+  __shared__ Best s_part[kWarps];               // this step's per-warp partial argmax
+  __shared__ __align__(8) Best s_inbox[2][kMaxCluster];  // every CTA's partial argmax, by step parity
+  __shared__ __align__(8) uint64_t s_ibar[2];   // completes when all partials of a step have arrived
+  __shared__ int2 s_dec[2];                     // (argmax, next node) of the step, by step parity
+  __shared__ int s_abort;
   __shared__ int s_wsum[kWarps];
   __shared__ int s_bad;
 
@@ -99,7 +122,13 @@ __global__ void __launch_bounds__(kThreads)
   const bool vec = (vocab % 4) == 0;  // rows then start 16-byte aligned (the base is checked on the host)
   if (tid == 0 && hi > lo) prefetch_l2(rows + lo, hi - lo);  // the root's row, while the tree is read
   // ---- the tree: tokens, parents (validated) and a children list per node
-  if (tid == 0) s_bad = 0;
+  if (tid == 0) {
+    s_bad = 0;
+    s_abort = 0;
+    mbar_init(&s_ibar[0], 1);
+    mbar_init(&s_ibar[1], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   for (int i = tid; i < num_nodes; i += kThreads) s_cur[i] = 0;
   __syncthreads();
   for (int i = tid; i < num_nodes; i += kThreads) {
@@ -142,7 +171,11 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
   }
-  // ---- the walk: per step one cluster barrier (partials visible cluster-wide) and two block barriers.
+  // every CTA's inbox barriers are initialised before the first remote store reaches them
+  cluster.sync();
+  // ---- the walk.  Per step: a block barrier for the warp partials; the CTA's partial is pushed into
+  // every CTA's inbox with st.async (completing bytes on the receiver's mbarrier); one warp waits for
+  // its own inbox, decides the next node, and a block barrier hands the decision to the CTA.
   int cur = 0, L = 0, a = 0;
   if (tid == 0) s_path[0] = 0;
   for (int step = 0;; ++step) {
@@ -189,27 +222,33 @@ __global__ void __launch_bounds__(kThreads)
     if (lane == 0) s_part[warp] = Best{bv, bid};
     __syncthreads();
     if (warp == 0) {
+      const int par = step & 1;
+      if (lane == 0) mbar_arrive_expect_tx(&s_ibar[par], static_cast<uint32_t>(C) * sizeof(Best));
       Best m = lane < kWarps ? s_part[lane] : Best{-INFINITY, INT_MAX};
-      warp_best(m.v, m.id);
-      if (lane == 0) s_slot[step & 1] = m;
-    }
-    cluster.sync();
-    if (warp == 0) {
-      // one warp per CTA gathers the cluster's partials and decides the next node
-      Best m{-INFINITY, INT_MAX};
-      if (lane < C) m = *cluster.map_shared_rank(&s_slot[step & 1], lane);
-      warp_best(m.v, m.id);
-      const int av = (m.id < 0 || m.id >= vocab) ? 0 : m.id;  // out of range only with NaN rows
+      warp_best(m.v, m.id);  // every lane holds the CTA's partial
+      if (lane < C)
+        st_async_best(cluster_addr(&s_inbox[par][rank], lane), m.v, m.id, cluster_addr(&s_ibar[par], lane));
+      // one warp per CTA waits for the cluster's partials and decides the next node
+      if (!warp_all_wait(&s_ibar[par], (step >> 1) & 1, &s_abort)) {
+        if (lane == 0) {
+          s_abort = 1;
+          report(status, JF_ERR_TIMEOUT);
+        }
+      }
+      Best g{-INFINITY, INT_MAX};
+      if (lane < C) g = s_inbox[par][lane];
+      warp_best(g.v, g.id);
+      const int av = (g.id < 0 || g.id >= vocab) ? 0 : g.id;  // out of range only with NaN rows
       // the child of cur carrying token av (the lowest index if several do)
       int mt = INT_MAX;
-      if (L < max_depth) {
+      if (L < max_depth && !s_abort) {
         for (int k = lane; k < nk; k += 32) {
           const int c = s_kid[k0 + k];
           if (s_tok[c] == av && c < mt) mt = c;
         }
       }
       mt = __reduce_min_sync(0xffffffffu, mt);
-      if (lane == 0) s_dec[step & 1] = make_int2(av, mt);
+      if (lane == 0) s_dec[par] = make_int2(av, mt);
     }
     __syncthreads();
     const int2 dec = s_dec[step & 1];
@@ -229,7 +268,7 @@ __global__ void __launch_bounds__(kThreads)
     int32_t* po = path + static_cast<long long>(b) * (max_depth + 1);
     for (int i = tid; i <= max_depth; i += kThreads) po[i] = (i <= L) ? s_path[i] : -1;
   }
-  // keep every CTA's shared memory alive until the last remote read of it has happened
+  // no CTA leaves while another may still write into its shared memory
   cluster.sync();
 }
 

@@ -26,6 +26,8 @@
 namespace jf {
 namespace build {
 
+__device__ const double g_exp2_frac32[32] = JF_EXP2_FRAC32;
+
 constexpr int kThreads = 256;
 constexpr int kPerThread = kStatsChunk / kThreads;  // 16
 constexpr int kSlots = kMaxDepths * kMaxTopk / 32;  // queue slots per lane (16)
@@ -114,12 +116,14 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ float s_max[kThreads / 32];
   __shared__ double s_sum[kThreads / 32];
   __shared__ Cand s_top[kThreads / 32][K];
+  __shared__ double s_tab[32];
   const int chunk = blockIdx.x, row = blockIdx.y;
   const int b = row / max_depth, d = row - b * max_depth;
   const float* x = logits + (static_cast<long long>(b) * depths + d) * vocab;
   const int lo = chunk * kStatsChunk;
   const int n = min(kStatsChunk, vocab - lo);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid < 32) s_tab[tid] = g_exp2_frac32[tid];  // visible after the barrier below
   float v[kPerThread];
   if (n == kStatsChunk && (reinterpret_cast<uintptr_t>(x + lo) & 15) == 0) {
     // full, 16-byte aligned chunk: thread t reads float4 number t, t + 256, ...
@@ -156,7 +160,7 @@ __global__ void __launch_bounds__(kThreads)
   for (int j = 0; j < kPerThread; ++j) {
     const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
     if (i < n) {
-      sum += exp_nonpos_f64(static_cast<double>(v[j]) - md);
+      sum += exp_nonpos_f64(static_cast<double>(v[j]) - md, s_tab);
       insert_k<K>(t, Cand{v[j], lo + i});
     }
   }
@@ -204,6 +208,7 @@ __device__ __forceinline__ double key_of_ord(unsigned long long o) {
 }
 
 struct ExpandSmem {
+  double tab[32];                       // 2^(j/32) for exp_nonpos_f64
   double lp[kMaxDepths + 1][kMaxTopk];  // lp[d][r], d = 1..max_depth
   int tok[kMaxDepths + 1][kMaxTopk];
   double key[kMaxBudget];  // sequential fallback: node keys
@@ -327,7 +332,8 @@ __device__ void expand_sequential(ExpandSmem& s, int lane, int max_depth, int to
 }
 
 // First position in [0, n) (n <= kMaxBudget) at which pred fails, for a pred that holds on a prefix;
-// R searches run interleaved (independent load chains), branch-free.
+// R searches run interleaved.  Branch-free: pred is always evaluated (on a clamped index) and must not
+// short-circuit -- divergent branches in these short searches cost several times the compares.
 template <int R, class Pred>
 __device__ __forceinline__ void prefix_lengths(int n, int (&cnt)[R], Pred pred) {
 #pragma unroll
@@ -336,7 +342,9 @@ __device__ __forceinline__ void prefix_lengths(int n, int (&cnt)[R], Pred pred) 
 #pragma unroll
     for (int i = 0; i < R; ++i) {
       const int t = cnt[i] + step;
-      if (t <= n && pred(i, t - 1)) cnt[i] = t;
+      const int jj = (t <= n ? t : n) - 1;  // in range; the outcome is discarded when t > n
+      const bool take = (t <= n) & pred(i, jj);
+      cnt[i] = take ? t : cnt[i];
     }
   }
 }
@@ -351,6 +359,8 @@ __global__ void __launch_bounds__(kExpandThreads)
   SelectSmem& q = *reinterpret_cast<SelectSmem*>(dyn);
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid < 32) s.tab[tid] = g_exp2_frac32[tid];
+  __syncthreads();
   // ---- 1. per-depth lse (float64) and top-k: one warp per depth, one lane per chunk partial
   for (int d = 1 + warp; d <= max_depth; d += kExpandThreads / 32) {
     const RowPartial* rp = part + (static_cast<long long>(b) * max_depth + (d - 1)) * nchunks;
@@ -363,7 +373,7 @@ __global__ void __launch_bounds__(kExpandThreads)
 #pragma unroll
     for (int i = 0; i < K; ++i) t[i] = Cand{-INFINITY, INT_MAX};
     for (int c = lane; c < nchunks; c += 32) {
-      sum += rp[c].sum * exp_nonpos_f64(static_cast<double>(rp[c].m) - md);
+      sum += rp[c].sum * exp_nonpos_f64(static_cast<double>(rp[c].m) - md, s.tab);
       Cand u[K];
 #pragma unroll
       for (int i = 0; i < K; ++i) u[i] = Cand{rp[c].val[i], rp[c].id[i]};
@@ -434,7 +444,7 @@ __global__ void __launch_bounds__(kExpandThreads)
       int cnt[K];
       prefix_lengths<K>(n_prev, cnt, [&](int r2, int jj) {
         const unsigned long long a = q.cord[r2][jj];
-        return a > kc || (a == kc && (jj < j || (jj == j && r2 < r)));
+        return (a > kc) | ((a == kc) & ((jj < j) | ((jj == j) & (r2 < r))));
       });
       int pos = 0;
 #pragma unroll
