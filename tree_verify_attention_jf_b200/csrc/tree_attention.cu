@@ -49,8 +49,8 @@ struct __align__(1024) Smem {
   uint8_t q[kAttnQTiles][kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
-  uint32_t anc[2][kMaxTreeNodes][kAncWords];
-  int par_stage[kMaxTreeNodes];  // the metadata warp's copy of the current segment's parent indices
+  uint32_t anc[kMaxTreeNodes][kAncWords];  // ancestor bitsets of the current segment's nodes
+  int jmp[kMaxTreeNodes];                   // pointer-jumping links while they are built
   long long cum_work[kMaxAttnBatch + 1];
   long long scan_warp[kThreads / 32];
   uint64_t bar_qfull, bar_qempty;
@@ -326,7 +326,7 @@ __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t 
 }
 
 // ------------------------------------------------------------------------------------------------
-// Warp 3: per-segment validation and ancestor bitsets
+// Warp 3: per-segment validation
 // ------------------------------------------------------------------------------------------------
 __device__ void metadata(Smem& s, const AttnParams& p, SegIter iter) {
   const int lane = threadIdx.x & 31;
@@ -368,10 +368,7 @@ __device__ void metadata(Smem& s, const AttnParams& p, SegIter iter) {
 #pragma unroll
     for (int k = 0; k < kMaxTreeNodes / 32; ++k) {
       const int i = lane + 32 * k;
-      if (i < g.N) {
-        if (pr[k] < -1 || pr[k] >= i) bad = 1;
-        s.par_stage[i] = (pr[k] >= i) ? -1 : pr[k];  // invalid parents are flagged; keep the walk in range
-      }
+      if (i < g.N && (pr[k] < -1 || pr[k] >= i)) bad = 1;
     }
     bad = __any_sync(0xffffffffu, bad);
     if (lane == 0) {
@@ -379,45 +376,6 @@ __device__ void metadata(Smem& s, const AttnParams& p, SegIter iter) {
       if (bad) report(p.status, JF_ERR_DEVICE_CHECK);
     }
     __syncwarp();
-    // --- ancestor bitsets (only needed when the segment reaches the tree slots).  Nodes are taken
-    // 32 at a time in index order; a node whose parent lies in an earlier chunk starts from the
-    // parent's finished bitset, the others resolve their in-chunk chain by pointer jumping over warp
-    // shuffles (5 rounds cover 32 levels).
-    if (static_cast<long long>(g.ke) * kBN > g.P) {
-      for (int base = 0; base < g.N; base += 32) {
-        const int i = base + lane;
-        uint32_t a[kAncWords];
-#pragma unroll
-        for (int w = 0; w < kAncWords; ++w) a[w] = 0u;
-        int jl = -1;  // lane of the next in-chunk ancestor still to merge
-        if (i < g.N) {
-          a[i >> 5] = 1u << (i & 31);
-          const int pi = s.par_stage[i];
-          if (pi >= 0 && pi < base) {
-#pragma unroll
-            for (int w = 0; w < kAncWords; ++w) a[w] |= s.anc[buf][pi][w];
-          } else if (pi >= base) {
-            jl = pi - base;
-          }
-        }
-#pragma unroll
-        for (int round = 0; round < 5; ++round) {
-          const int src = jl >= 0 ? jl : lane;
-#pragma unroll
-          for (int w = 0; w < kAncWords; ++w) {
-            const uint32_t o = __shfl_sync(0xffffffffu, a[w], src);
-            if (jl >= 0) a[w] |= o;
-          }
-          const int oj = __shfl_sync(0xffffffffu, jl, src);
-          jl = jl >= 0 ? oj : -1;
-        }
-        if (i < g.N) {
-#pragma unroll
-          for (int w = 0; w < kAncWords; ++w) s.anc[buf][i][w] = a[w];
-        }
-        __syncwarp();
-      }
-    }
     __threadfence_block();
     mbar_arrive(&s.bar_metafull[buf]);
     ++sidx;
@@ -473,6 +431,53 @@ __device__ __forceinline__ float4* part_ptr(const AttnParams& p, int slot, int c
   return reinterpret_cast<float4*>(p.part_o) + (static_cast<long long>(slot) * 32 + c4) * kBM + r;
 }
 
+// Named barrier 1 joins the 256 softmax threads (warps 4-11).
+__device__ __forceinline__ void softmax_bar() { named_bar_sync(1, 2 * kBM); }
+__device__ __forceinline__ bool softmax_bar_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(2 * kBM)
+      : "memory");
+  return r != 0;
+}
+
+// Ancestor bitsets (node itself included) of the segment's sequence, one softmax thread per node, by
+// pointer jumping: anc[i] covers the path from i up to (not including) jmp[i]; each round merges the
+// set at jmp[i] and jumps there, so a tree of depth D needs ceil(log2 D) + 1 rounds.  Parents outside
+// [-1, i) are treated as -1 (the metadata warp flags such a sequence, whose output is not stored).
+__device__ bool build_ancestors(Smem& s, const AttnParams& p, const Seg& g) {
+  const int i = static_cast<int>(threadIdx.x) - 128;  // 0 .. 255
+  softmax_bar();  // every read of the previous segment's bitsets is done
+  int pj = -1;
+  if (i < g.N) {
+    const int pi = __ldg(p.parent + g.off + i);
+    pj = (pi >= 0 && pi < i) ? pi : -1;
+#pragma unroll
+    for (int w = 0; w < kAncWords; ++w) s.anc[i][w] = (w == (i >> 5)) ? (1u << (i & 31)) : 0u;
+    s.jmp[i] = pj;
+  }
+  for (int round = 0; softmax_bar_or(pj >= 0); ++round) {
+    if (round > kMaxTreeNodes) return false;  // unreachable for valid input; keeps the loop bounded
+    uint32_t add[kAncWords];
+    int nj = -1;
+    if (pj >= 0) {
+#pragma unroll
+      for (int w = 0; w < kAncWords; ++w) add[w] = s.anc[pj][w];
+      nj = s.jmp[pj];
+    }
+    softmax_bar();  // all reads of this round before any write
+    if (pj >= 0) {
+#pragma unroll
+      for (int w = 0; w < kAncWords; ++w) s.anc[i][w] |= add[w];
+      s.jmp[i] = nj;
+      pj = nj;
+    }
+  }
+  return true;
+}
+
 __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uint32_t tmem, int qt) {
   const int r = threadIdx.x - 128 - qt * kBM;  // row of M tile qt == TMEM lane
   const int wq = (threadIdx.x >> 5) & 3;
@@ -489,15 +494,11 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
     const int node = (g.mp * kAttnQTiles + qt) * nodes_per_tile + r / p.group;
     const int head = g.kvh * p.group + (r % p.group);
     const bool row_valid = node < g.N;
-    const uint32_t* anc = &s.anc[buf][row_valid ? node : 0][0];
+    if (static_cast<long long>(g.ke) * kBN > g.P && !build_ancestors(s, p, g)) return set_abort(s, p);
+    const uint32_t* anc = &s.anc[row_valid ? node : 0][0];
     float m_use = -INFINITY, l = 0.f;
-    bool meta_seen = false;
     for (int t = g.kb; t < g.ke; ++t, ++it) {
       const bool tree_tile = (t + 1) * kBN > g.P;
-      if (tree_tile && !meta_seen) {
-        if (!warp_wait(&s.bar_metafull[buf], (sidx >> 1) & 1, abort)) return set_abort(s, p);
-        meta_seen = true;
-      }
       if (!warp_wait(&s.bar_sfull[qt], it & 1, abort)) return set_abort(s, p);
       // S_qt(it) ready also means PV_qt(it-1) is complete: its commit tracks every earlier MMA.
       tc_fence_after();
@@ -588,9 +589,7 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
       mbar_arrive(&s.bar_pfull[qt]);
     }
     // ---------------- epilogue of the segment
-    if (!meta_seen) {
-      if (!warp_wait(&s.bar_metafull[buf], (sidx >> 1) & 1, abort)) return set_abort(s, p);
-    }
+    if (!warp_wait(&s.bar_metafull[buf], (sidx >> 1) & 1, abort)) return set_abort(s, p);
     const bool seg_ok = s.meta_valid[buf] != 0;
     if (!warp_wait(&s.bar_pvdone[qt], (it - 1) & 1, abort)) return set_abort(s, p);
     tc_fence_after();
@@ -746,12 +745,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------------------------------------
 constexpr int kCombineThreads = 256;
 constexpr int kCombineRows = 32;
-constexpr int kCombineQuads = 4;  // 4-column groups per thread
+constexpr int kCombineQuads = 4;  // 4-column groups per thread (a block covers 32 rows x 32 * kCombineQuads columns)
 constexpr int kSegBatch = 4;      // segments whose partials are loaded in one batch
-constexpr int kItemsPerUnit = kAttnQTiles * (kBM / kCombineRows);
+constexpr int kColParts = 128 / (4 * kCombineQuads * (kCombineThreads / 32));  // column parts of a 32-row block
+constexpr int kItemsPerUnit = kAttnQTiles * (kBM / kCombineRows) * kColParts;
 
 __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnParams p, int ncta) {
   static_assert(kMaxGrid <= kCombineThreads, "one descriptor slot per thread");
+  static_assert(kColParts >= 1 && kColParts * 4 * kCombineQuads * (kCombineThreads / 32) == 128, "column split");
   __shared__ int4 s_desc[kMaxGrid];
   __shared__ int s_c0[kMaxGrid];
   __shared__ int s_wcount[kCombineThreads / 32];
@@ -780,12 +781,13 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
   const int s_n = total;
   const int n_items = s_n * kItemsPerUnit;
   const int rl = lane;
-  const int q0 = warp * kCombineQuads;  // first 4-column group of this thread
   const int nodes_per_tile = kBM / p.group;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int u = item / kItemsPerUnit;
-    const int qt = (item / (kBM / kCombineRows)) % kAttnQTiles;
-    const int rb = item % (kBM / kCombineRows);
+    const int cp = item % kColParts;
+    const int qt = (item / (kColParts * (kBM / kCombineRows))) % kAttnQTiles;
+    const int rb = (item / kColParts) % (kBM / kCombineRows);
+    const int q0 = (cp * (kCombineThreads / 32) + warp) * kCombineQuads;  // first 4-column group of this thread
     const int4 d = s_desc[u];
     const int c0 = s_c0[u], c1 = d.x;
     const int r = rb * kCombineRows + rl;  // row of the M tile
@@ -845,18 +847,10 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
     }
     if (!ok) continue;
     const float inv = 1.f / L;
-    uint4 o[2];
-    o[0].x = pack_bf16x2(acc[0].x * inv, acc[0].y * inv);
-    o[0].y = pack_bf16x2(acc[0].z * inv, acc[0].w * inv);
-    o[0].z = pack_bf16x2(acc[1].x * inv, acc[1].y * inv);
-    o[0].w = pack_bf16x2(acc[1].z * inv, acc[1].w * inv);
-    o[1].x = pack_bf16x2(acc[2].x * inv, acc[2].y * inv);
-    o[1].y = pack_bf16x2(acc[2].z * inv, acc[2].w * inv);
-    o[1].z = pack_bf16x2(acc[3].x * inv, acc[3].y * inv);
-    o[1].w = pack_bf16x2(acc[3].z * inv, acc[3].w * inv);
-    uint4* dst = reinterpret_cast<uint4*>(p.out + grow * 128 + q0 * 4);
-    dst[0] = o[0];
-    dst[1] = o[1];
+    uint2* dst = reinterpret_cast<uint2*>(p.out + grow * 128 + q0 * 4);
+#pragma unroll
+    for (int q = 0; q < kCombineQuads; ++q)
+      dst[q] = make_uint2(pack_bf16x2(acc[q].x * inv, acc[q].y * inv), pack_bf16x2(acc[q].z * inv, acc[q].w * inv));
     if (q0 == 0 && p.lse != nullptr) p.lse[grow] = (M + __log2f(L)) * 0.69314718055994531f;
   }
 }
