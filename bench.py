@@ -34,17 +34,22 @@ WORKLOADS = {
     "qwen3_8b": dict(batch=1, hq=32, hkv=8, prefix=4096, budget=256, topk=4, max_depth=16, vocab=151936, depths=16),
     "qwen3_30b_a3b": dict(batch=4, hq=32, hkv=4, prefix=32768, budget=256, topk=4, max_depth=16, vocab=151936,
                           depths=16),
-    "serving": dict(batch=16, hq=32, hkv=8, prefix=4608, budget=64, topk=4, max_depth=12, vocab=151936, depths=16),
+    # serving: per-sequence prefix lengths uniform in [1024, 8192], all pages of the batch interleaved in one pool
+    "serving": dict(batch=16, hq=32, hkv=8, prefix=(1024, 8192), budget=64, topk=4, max_depth=12, vocab=151936,
+                    depths=16),
 }
 HEAD_DIM = 128
 PAGE = 16
 L2_FLUSH_BYTES = 256 << 20
 LAUNCHES_PER_STEP = 5
-# DRAM traffic of one tree_attention_kernel launch on the default workload (dram__bytes_read.sum +
-# dram__bytes_write.sum from the capture summarised in profiles/tree_attention_kernel_qwen3_8b.md), valid
+# DRAM traffic of one tree_attention_kernel launch per workload (dram__bytes_read.sum + dram__bytes_write.sum
+# from the captures summarised in profiles/tree_attention_kernel_*.md and profiles/serving_kernels.md), valid
 # only for the kernel source it was taken on: the roofline reports null once that source has changed.
-ATTN_TRAFFIC = {"qwen3_8b": {"bytes": 20.014080e6 + 0.014848e6,
-                             "source_sha256": "3245e97978596ad4eab819431ec28bc46815ea6653a257a672b238bf5c828868"}}
+ATTN_TRAFFIC = {
+    "qwen3_8b": {"bytes": 20.009984e6 + 0.030464e6, "source_sha256": "c67f5208c48f9964917b2e865dab918a35ada932c8750fb2c19c2da8118645ee"},
+    "qwen3_30b_a3b": {"bytes": 2.155419e9 + 0.022077e9, "source_sha256": "c67f5208c48f9964917b2e865dab918a35ada932c8750fb2c19c2da8118645ee"},
+    "serving": {"bytes": 321.87264e6 + 19.57376e6, "source_sha256": "c67f5208c48f9964917b2e865dab918a35ada932c8750fb2c19c2da8118645ee"},
+}
 
 
 def peaks():
@@ -59,13 +64,21 @@ def peaks():
 # ----------------------------------------------------------------------------------------------
 # Inputs (seeded, synthetic; shapes of the pages' Qwen3 workloads)
 # ----------------------------------------------------------------------------------------------
+def prefix_lengths(cfg, rng):
+    """Per-sequence prefix lengths: fixed, or uniform over a (low, high) range."""
+    B, pr = cfg["batch"], cfg["prefix"]
+    if isinstance(pr, tuple):
+        return [int(x) for x in rng.integers(pr[0], pr[1] + 1, size=B)]
+    return [int(pr)] * B
+
+
 def make_inputs(cfg, seed):
     from tree_verify_attention_jf_b200 import synth
 
     B, N = cfg["batch"], cfg["budget"]
     rng = np.random.default_rng(seed)
     x, roots = synth.draft_logits(seed, B, cfg["depths"], cfg["vocab"])
-    prefix = [cfg["prefix"]] * B
+    prefix = prefix_lengths(cfg, rng)
     pages_per_seq = [(P + N + PAGE - 1) // PAGE for P in prefix]
     bt, num_pages = synth.page_pool(rng, pages_per_seq, interleave=True)
     q = rng.standard_normal((B * N, cfg["hq"], HEAD_DIM), dtype=np.float32) * np.float32(0.5)
@@ -85,6 +98,22 @@ def attention_traffic(workload):
     with open(src, "rb") as f:
         digest = hashlib.sha256(f.read()).hexdigest()
     return rec["bytes"] if digest == rec["source_sha256"] else None
+
+
+# Workloads whose attention is bandwidth-bound (arithmetic intensity at or below the ridge) are graded
+# against HBM bandwidth, the others against the dense bf16 tensor peak.
+HBM_BOUND = {"serving"}
+
+
+def roofline(workload, tflops, gbs, pk, flops, nbytes):
+    common = {"kernel": "jf_tree_attention (tree_attention_kernel + combine_kernel)",
+              "traffic": attention_traffic(workload), "algorithmic_flops": flops, "algorithmic_bytes": nbytes}
+    if workload in HBM_BOUND:
+        return dict(common, bound="hbm", achieved=gbs, peak=pk["hbm"], unit="GB/s", frac=gbs / pk["hbm"],
+                    peak_source=pk["src"] + " HBM copy", tensor_achieved_tflops=tflops,
+                    tensor_frac=tflops / pk["bf16"])
+    return dict(common, bound="tensor", achieved=tflops, peak=pk["bf16"], unit="TFLOP/s", frac=tflops / pk["bf16"],
+                peak_source=pk["src"] + " bf16 burst", hbm_achieved_gbs=gbs, hbm_frac=gbs / pk["hbm"])
 
 
 def rank_seed(rank):
@@ -314,7 +343,7 @@ def run_gpu(args, cfg, rank, world, device):
     h2d = draft_h.numel() * 4 + q_h.numel() * 2 + tgt_h.numel() * 4
     d2h = res_h.numel() * 4
     return dict(step_ms=step_ms, attn_ms=attn_ms, build_ms=build_ms, accept_ms=accept_ms, clocks=clocks,
-                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, parent=par_h)
+                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, parent=par_h, prefix=inp["prefix"])
 
 
 def barrier(world):
@@ -348,7 +377,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", 0))
     metric = "tree nodes verified/sec"
     config = {"workload": f"{args.workload}_tree_verify", "batch": cfg["batch"], "q_heads": cfg["hq"],
-              "kv_heads": cfg["hkv"], "head_dim": HEAD_DIM, "prefix": cfg["prefix"], "page_size": PAGE,
+              "kv_heads": cfg["hkv"], "head_dim": HEAD_DIM,
+              "prefix": (f"U[{cfg['prefix'][0]},{cfg['prefix'][1]}]" if isinstance(cfg["prefix"], tuple)
+                         else cfg["prefix"]), "page_size": PAGE,
               "budget": cfg["budget"], "topk": cfg["topk"], "max_depth": cfg["max_depth"], "vocab": cfg["vocab"],
               "step": "build_tree + tree_attention (one layer) + accept", "parallelism": f"replicas{world}",
               "l2": "flushed between steps (256 MiB write outside the timed events)",
@@ -381,11 +412,12 @@ def main():
     attn_ms = statistics.mean(r["attn_ms"])
     B, N = cfg["batch"], cfg["budget"]
     pk = peaks()
-    pairs = visible_pairs(r["parent"], [cfg["prefix"]] * B)
+    prefixes = [int(x) for x in r["prefix"]]
+    pairs = visible_pairs(r["parent"], prefixes)
     flops = 4.0 * HEAD_DIM * cfg["hq"] * pairs
-    kv_bytes = B * cfg["hkv"] * (cfg["prefix"] + N) * HEAD_DIM * 2 * 2
+    kv_bytes = sum(cfg["hkv"] * (P + N) * HEAD_DIM * 2 * 2 for P in prefixes)
     qo_bytes = 2 * B * N * cfg["hq"] * HEAD_DIM * 2
-    meta_bytes = B * (4 * (cfg["prefix"] + N + PAGE - 1) // PAGE + 4 * N + 12)
+    meta_bytes = sum(4 * ((P + N + PAGE - 1) // PAGE) + 4 * N + 12 for P in prefixes)
     tflops = flops / (attn_ms * 1e-3) / 1e12
     gbs = (kv_bytes + qo_bytes + meta_bytes) / (attn_ms * 1e-3) / 1e9
     shares = {"build_tree": statistics.mean(r["build_ms"]) / mean_step,
@@ -404,12 +436,7 @@ def main():
         "metric": metric, "value": job_nodes_per_sec(B, N, world, step_ms), "unit": "nodes/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)", "config": config,
-        "roofline": {"kernel": "jf_tree_attention (tree_attention_kernel + combine_kernel)", "bound": "tensor",
-                     "achieved": tflops, "peak": pk["bf16"], "unit": "TFLOP/s", "frac": tflops / pk["bf16"],
-                     "traffic": attention_traffic(args.workload),
-                     "peak_source": pk["src"] + " bf16 burst",
-                     "hbm_achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm"],
-                     "algorithmic_flops": flops, "algorithmic_bytes": kv_bytes + qo_bytes + meta_bytes},
+        "roofline": roofline(args.workload, tflops, gbs, pk, flops, kv_bytes + qo_bytes + meta_bytes),
         "kernel_ms": {"build_tree": statistics.mean(r["build_ms"]), "tree_attention": attn_ms,
                       "accept": statistics.mean(r["accept_ms"])},
         "time_share": shares,
