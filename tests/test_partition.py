@@ -1,12 +1,17 @@
 """Host-side model of the attention kernel's stream-K partition (the same integer formulas as the
 device plan): every (unit, kv tile) pair is covered exactly once, a unit's sharing CTAs are exactly
-those whose range intersects it, partial slots never collide, and every CTA's range is non-empty."""
+those that hold one of its kv tiles, partial slots never collide, every CTA's range is non-empty, and
+a CTA that starts segments in mid-range gets correspondingly fewer kv tiles.
+
+Each unit costs SEG_COST + kt positions: SEG_COST leading positions (the price of starting a segment
+in mid-kernel) and then its kt kv tiles."""
 import itertools
 
 import numpy as np
 import pytest
 
 BN, BM = 128, 128
+SEG_COST = 3
 
 
 def plan(prefix, nodes, hkv, group):
@@ -17,7 +22,7 @@ def plan(prefix, nodes, hkv, group):
             continue
         kt = (P + N + BN - 1) // BN
         mt = (N * group + BM - 1) // BM
-        work.append(hkv * mt * kt)
+        work.append(hkv * mt * (kt + SEG_COST))
     cum = np.concatenate([[0], np.cumsum(work)]).astype(np.int64)
     return cum
 
@@ -38,15 +43,18 @@ def segments(prefix, nodes, hkv, group, grid):
             P, N = prefix[b], nodes[b]
             kt = (P + N + BN - 1) // BN
             mtn = (N * group + BM - 1) // BM
-            local = x - cum[b]
-            unit = local // kt
-            kb = local - unit * kt
-            u0, u1 = cum[b] + unit * kt, cum[b] + unit * kt + kt
+            span = kt + SEG_COST
+            unit = (x - cum[b]) // span
+            u0, u1 = cum[b] + unit * span, cum[b] + unit * span + span
             e = min(xend, u1)
-            c0, c1 = cta_of(u0), cta_of(u1 - 1)
-            slot = 2 * c + 1 if c == c0 else 2 * c
-            out.append(dict(cta=c, b=b, kvh=unit // mtn, mt=unit % mtn, kb=kb, ke=kb + (e - x), c0=c0, c1=c1, slot=slot))
+            t0, t1 = x - u0 - SEG_COST, e - u0 - SEG_COST
             x = e
+            if t1 <= 0:
+                continue
+            c0, c1 = cta_of(u0 + SEG_COST), cta_of(u1 - 1)
+            slot = 2 * c + 1 if c == c0 else 2 * c
+            out.append(dict(cta=c, b=b, kvh=unit // mtn, mt=unit % mtn, kb=max(t0, 0), ke=t1, c0=c0, c1=c1,
+                            slot=slot, range=(c * W // G, (c + 1) * W // G)))
     return out, W, G
 
 
@@ -66,7 +74,17 @@ def test_cover_exactly_once(prefix, nodes, hkv, group, grid):
             key = (s["b"], s["kvh"], s["mt"], t)
             assert key not in seen
             seen[key] = s["cta"]
-    assert len(seen) == W
+    tiles = sum(hkv * ((N * group + BM - 1) // BM) * ((P + N + BN - 1) // BN)
+                for P, N in zip(prefix, nodes) if N > 0)
+    assert len(seen) == tiles
+    assert W == tiles + SEG_COST * sum(hkv * ((N * group + BM - 1) // BM) for N in nodes if N > 0)
+    per_cta = {}
+    for s in segs:
+        per_cta.setdefault(s["cta"], []).append(s)
+    for c, ss in per_cta.items():
+        lo, hi = ss[0]["range"]
+        real = sum(x["ke"] - x["kb"] for x in ss)
+        assert real + SEG_COST * (len(ss) - 1) <= hi - lo
     units = {}
     for s in segs:
         units.setdefault((s["b"], s["kvh"], s["mt"]), []).append(s)

@@ -21,8 +21,8 @@
 //     8-11 (one thread per row of M tile 0 / 1) run the online softmax out of TMEM with a lazy rescale
 //     of O, and the epilogue.
 //   * The tree mask only touches tiles that hold tree slots; prefix tiles are unmasked.
-//   * Work split: the flattened (unit, kv tile) space is cut into equal contiguous ranges, one per CTA
-//     (stream-K).  A unit cut between CTAs writes fp32 partials (O, running max, row sum) and its
+//   * Work split: the flattened (unit, kv tile) space, in which every unit also carries a fixed cost for
+//     the segment start, is cut into equal contiguous ranges, one per CTA (stream-K).  A unit cut between CTAs writes fp32 partials (O, running max, row sum) and its
 //     first CTA records the unit in a descriptor slot; combine_kernel, launched right behind on the
 //     same stream with a programmatic dependency, merges each recorded unit's partials and stores the
 //     bf16 output.  Nothing spins on another CTA.
@@ -43,7 +43,8 @@ constexpr int kTileBytes = 2 * kHalfBytes;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmS = 0;    // S_i at column 128 * i
 constexpr uint32_t kTmO = 256;  // O_i at column 256 + 128 * i
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow up to 2^8 before O is rescaled
+constexpr float kRescaleThreshold = 8.0f;
+constexpr int kSegCost = 3;  // kv tiles' worth of time that starting a segment in mid-kernel costs  // log2 units: P may grow up to 2^8 before O is rescaled
 
 struct __align__(1024) Smem {
   uint8_t q[kAttnQTiles][kTileBytes];
@@ -52,6 +53,8 @@ struct __align__(1024) Smem {
   uint32_t anc[kMaxTreeNodes][kAncWords];  // ancestor bitsets of the current segment's nodes
   int jmp[kMaxTreeNodes];                   // pointer-jumping links while they are built
   long long cum_work[kMaxAttnBatch + 1];
+  int seq_p[kMaxAttnBatch];       // prefix length of every sequence (copied once by the plan)
+  int seq_off[kMaxAttnBatch + 1]; // tree_offsets
   long long scan_warp[kThreads / 32];
   uint64_t bar_qfull, bar_qempty;
   uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
@@ -79,31 +82,40 @@ __device__ __forceinline__ int pairs_of(int N, int group) {
   return (mtn + kAttnQTiles - 1) / kAttnQTiles;
 }
 
+// Cost space: a unit costs kSegCost + kt, its kv tiles preceded by kSegCost positions that stand for
+// the time a CTA loses when it starts a segment in mid-kernel (the previous segment's epilogue, the Q
+// reload, the refill of the K/V pipeline).  Cutting this space into equal ranges gives a CTA that
+// crosses a unit boundary correspondingly fewer kv tiles.  A CTA whose range ends inside a unit's
+// leading positions takes no part in that unit.
 struct SegIter {
   long long x, xend, W;
   int G, b;
   __device__ bool next(const Smem& s, const AttnParams& p, Seg& g) {
-    if (x >= xend) return false;
-    while (s.cum_work[b + 1] <= x) ++b;
-    g.b = b;
-    g.P = p.prefix_lens[b];
-    g.off = p.tree_offsets[b];
-    g.N = p.tree_offsets[b + 1] - g.off;
-    g.kt = (g.P + g.N + kBN - 1) / kBN;
-    const int mpn = pairs_of(g.N, p.group);
-    const long long local = x - s.cum_work[b];
-    const long long unit = local / g.kt;
-    g.kb = static_cast<int>(local - unit * g.kt);
-    g.kvh = static_cast<int>(unit / mpn);
-    g.mp = static_cast<int>(unit - static_cast<long long>(g.kvh) * mpn);
-    const long long u0 = s.cum_work[b] + unit * g.kt, u1 = u0 + g.kt;
-    const long long e = xend < u1 ? xend : u1;
-    g.ke = g.kb + static_cast<int>(e - x);
-    g.c0 = cta_of(u0, W, G);
-    g.c1 = cta_of(u1 - 1, W, G);
-    g.slot = (static_cast<int>(blockIdx.x) == g.c0) ? 2 * blockIdx.x + 1 : 2 * blockIdx.x;
-    x = e;
-    return true;
+    while (x < xend) {
+      while (s.cum_work[b + 1] <= x) ++b;
+      g.b = b;
+      g.P = s.seq_p[b];
+      g.off = s.seq_off[b];
+      g.N = s.seq_off[b + 1] - g.off;
+      g.kt = (g.P + g.N + kBN - 1) / kBN;
+      const long long span = g.kt + kSegCost;
+      const int mpn = pairs_of(g.N, p.group);
+      const long long unit = (x - s.cum_work[b]) / span;
+      const long long u0 = s.cum_work[b] + unit * span, u1 = u0 + span;
+      const long long e = xend < u1 ? xend : u1;
+      const long long t0 = x - u0 - kSegCost, t1 = e - u0 - kSegCost;  // kv tiles [t0, t1) of the unit
+      x = e;
+      if (t1 <= 0) continue;
+      g.kb = t0 < 0 ? 0 : static_cast<int>(t0);
+      g.ke = static_cast<int>(t1);
+      g.kvh = static_cast<int>(unit / mpn);
+      g.mp = static_cast<int>(unit - static_cast<long long>(g.kvh) * mpn);
+      g.c0 = cta_of(u0 + kSegCost, W, G);  // owner of the unit's first kv tile
+      g.c1 = cta_of(u1 - 1, W, G);         // owner of its last
+      g.slot = (static_cast<int>(blockIdx.x) == g.c0) ? 2 * blockIdx.x + 1 : 2 * blockIdx.x;
+      return true;
+    }
+    return false;
   }
 };
 
@@ -120,7 +132,7 @@ __device__ __forceinline__ void set_abort(Smem& s, const AttnParams& p) {
 }
 
 // ------------------------------------------------------------------------------------------------
-// Plan: per-sequence work (kv heads x M-tile pairs x kv tiles), exclusive prefix sum in shared memory,
+// Plan: per-sequence cost (kv heads x M-tile pairs x (kv tiles + kSegCost)), exclusive prefix sum in shared memory,
 // validation of the batch-level metadata.  Every CTA computes the same plan.
 // ------------------------------------------------------------------------------------------------
 __device__ void build_plan(Smem& s, const AttnParams& p) {
@@ -133,16 +145,20 @@ __device__ void build_plan(Smem& s, const AttnParams& p) {
   if (tid == 0) s.bad_meta = 0;
   __syncthreads();
   if (tid == 0 && (p.tree_offsets[0] != 0 || p.tree_offsets[B] != p.total_nodes)) bad = 1;
+  if (tid == 0) s.seq_off[B] = p.tree_offsets[B];
   for (int b = b0; b < b0 + per && b < B; ++b) {
     const int P = p.prefix_lens[b];
-    const int N = p.tree_offsets[b + 1] - p.tree_offsets[b];
+    const int off = p.tree_offsets[b];
+    const int N = p.tree_offsets[b + 1] - off;
+    s.seq_p[b] = P;
+    s.seq_off[b] = off;
     if (P < 0 || N < 0 || N > kMaxTreeNodes) {
       bad = 1;
       continue;
     }
     if (N == 0) continue;
     const long long kt = (static_cast<long long>(P) + N + kBN - 1) / kBN;
-    local += static_cast<long long>(p.hkv) * pairs_of(N, p.group) * kt;
+    local += static_cast<long long>(p.hkv) * pairs_of(N, p.group) * (kt + kSegCost);
   }
   if (bad) atomicOr(&s.bad_meta, 1);
   long long incl = local;
@@ -157,11 +173,11 @@ __device__ void build_plan(Smem& s, const AttnParams& p) {
   long long run = warp_off + incl - local;
   for (int b = b0; b < b0 + per && b < B; ++b) {
     s.cum_work[b] = run;
-    const int P = p.prefix_lens[b];
-    const int N = p.tree_offsets[b + 1] - p.tree_offsets[b];
+    const int P = s.seq_p[b];
+    const int N = s.seq_off[b + 1] - s.seq_off[b];
     if (P < 0 || N <= 0 || N > kMaxTreeNodes) continue;
     const long long kt = (static_cast<long long>(P) + N + kBN - 1) / kBN;
-    run += static_cast<long long>(p.hkv) * pairs_of(N, p.group) * kt;
+    run += static_cast<long long>(p.hkv) * pairs_of(N, p.group) * (kt + kSegCost);
   }
   if (tid == kThreads - 1) s.cum_work[B] = run;
   __syncthreads();
@@ -180,16 +196,6 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
   uint32_t it = 0, sidx = 0;
   const int nodes_per_tile = kBM / p.group;
   while (iter.next(s, p, g)) {
-    if (!is_v) {
-      if (!warp_wait(&s.bar_qempty, (sidx & 1) ^ 1, abort)) return set_abort(s, p);
-      if (lane == 0) mbar_arrive_expect_tx(&s.bar_qfull, kAttnQTiles * kTileBytes);
-      __syncwarp();
-      if (lane < 2 * kAttnQTiles) {  // lane: Q tile lane / 2, half lane % 2
-        const int qt = lane >> 1, half = lane & 1;
-        const int node0 = g.off + (g.mp * kAttnQTiles + qt) * nodes_per_tile;
-        tma_load_3d(s.q[qt] + half * kHalfBytes, tm_q, &s.bar_qfull, half * 64, g.kvh * p.group, node0);
-      }
-    }
     const int npg = (g.P + g.N + kPage - 1) / kPage;
     const int32_t* bt = p.block_table + static_cast<long long>(g.b) * p.max_pages;
     // Page ids are fetched four tiles at a time (lane l: logical page 8 * (t0 + l / 8) + l % 8, -1 = not
@@ -208,6 +214,17 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
     };
     int ids_cur = batch_ids(g.kb);
     int ids_next = batch_ids(g.kb + 4);
+    // the Q tiles go out while the page ids are on their way
+    if (!is_v) {
+      if (!warp_wait(&s.bar_qempty, (sidx & 1) ^ 1, abort)) return set_abort(s, p);
+      if (lane == 0) mbar_arrive_expect_tx(&s.bar_qfull, kAttnQTiles * kTileBytes);
+      __syncwarp();
+      if (lane < 2 * kAttnQTiles) {  // lane: Q tile lane / 2, half lane % 2
+        const int qt = lane >> 1, half = lane & 1;
+        const int node0 = g.off + (g.mp * kAttnQTiles + qt) * nodes_per_tile;
+        tma_load_3d(s.q[qt] + half * kHalfBytes, tm_q, &s.bar_qfull, half * 64, g.kvh * p.group, node0);
+      }
+    }
     for (int t = g.kb; t < g.ke; ++t, ++it) {
       const int st = it % kStages;
       const uint32_t ph = (it / kStages) & 1;
@@ -651,30 +668,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // has finished, but it no longer pays a launch after the last CTA exits.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  build_plan(s, p);
-  if (s.bad_meta) {
-    if (blockIdx.x == 0 && tid == 0) report(p.status, JF_ERR_DEVICE_CHECK);
-    return;
-  }
-  const long long W = s.cum_work[p.batch];
-  if (W <= 0) return;
-  const int G = static_cast<int>(W < static_cast<long long>(gridDim.x) ? W : static_cast<long long>(gridDim.x));
-  if (static_cast<int>(blockIdx.x) >= G) return;
-  SegIter iter;
-  iter.x = static_cast<long long>(blockIdx.x) * W / G;
-  iter.xend = static_cast<long long>(blockIdx.x + 1) * W / G;
-  iter.W = W;
-  iter.G = G;
-  {
-    // first sequence touched by this CTA: binary search over cum_work
-    int lo = 0, hi = p.batch - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s.cum_work[mid] <= iter.x) lo = mid; else hi = mid - 1;
-    }
-    iter.b = lo;
-  }
-
+  // Everything that does not depend on the plan is started before it, so that its latency (cold
+  // descriptor and tensor-memory setup) hides behind the plan's metadata loads: the barriers, the
+  // tensor-map prefetches and the TMEM allocation.  The plan's barriers publish all of it.
   if (tid == 0) {
     mbar_init(&s.bar_qfull, 1);
     mbar_init(&s.bar_qempty, 1);
@@ -706,9 +702,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  build_plan(s, p);
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
+  bool idle = s.bad_meta != 0;
+  if (idle && blockIdx.x == 0 && tid == 0) report(p.status, JF_ERR_DEVICE_CHECK);
+  const long long W = s.cum_work[p.batch];
+  const int G = static_cast<int>(W < static_cast<long long>(gridDim.x) ? W : static_cast<long long>(gridDim.x));
+  idle = idle || W <= 0 || static_cast<int>(blockIdx.x) >= G;
+  if (idle) {  // uniform over the CTA
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    return;
+  }
+  SegIter iter;
+  iter.x = static_cast<long long>(blockIdx.x) * W / G;
+  iter.xend = static_cast<long long>(blockIdx.x + 1) * W / G;
+  iter.W = W;
+  iter.G = G;
+  {
+    // first sequence touched by this CTA: binary search over cum_work
+    int lo = 0, hi = p.batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s.cum_work[mid] <= iter.x) lo = mid; else hi = mid - 1;
+    }
+    iter.b = lo;
+  }
 
   // Register split (the launch gives every thread 168): the copy/MMA/metadata warpgroup runs on 80,
   // which lets the two softmax warpgroups hold a whole 128-column row of S in registers (208).
