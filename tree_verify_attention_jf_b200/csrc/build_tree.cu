@@ -6,7 +6,8 @@
 //
 // Kernel 1 (row statistics, HBM-bound): one CTA per (row, 4096-entry chunk) of the [B, depths, V]
 // logits reads its chunk once (16-byte loads when the rows allow), and writes the chunk max, the
-// float64 sum of exp(x - chunk max) and the chunk's top-8 by (logit desc, id asc).
+// float64 sum of exp(x - chunk max) and the chunk's top-8 by (logit desc, id asc).  Only elements at
+// or above a per-warp bound (the K-th largest lane maximum) enter the sorted top-K insertion.
 // Kernel 2 (expansion, one CTA per sequence): merges the chunk partials into lse and the top-k per
 // depth (float64), then selects the budget's nodes.  Best-first popping by (key desc, depth asc,
 // parent index asc, rank asc) yields the budget-1 first nodes of that total order, so the kernel
@@ -104,6 +105,20 @@ __device__ __forceinline__ float warp_max_f(float x) {
   return x;
 }
 
+// A lower bound on the K-th largest of the warp's 32 values: K rounds of "take the warp max, drop every
+// lane that holds it".  Ties are dropped together, so the result is the K-th largest distinct value
+// (or -inf if there are fewer), which never exceeds the K-th largest counted with multiplicity.
+template <int K>
+__device__ __forceinline__ float warp_kth_bound(float x) {
+  float m = -INFINITY;
+#pragma unroll
+  for (int r = 0; r < K; ++r) {
+    m = warp_max_f(x);
+    if (x == m) x = -INFINITY;
+  }
+  return m;
+}
+
 // ------------------------------------------------------------------------------------------------
 // Kernel 1: chunk statistics.  grid = (chunks, batch * max_depth)
 // ------------------------------------------------------------------------------------------------
@@ -142,10 +157,13 @@ __global__ void __launch_bounds__(kThreads)
       v[j] = (i < n) ? __ldg(x + lo + i) : -INFINITY;
     }
   }
-  float m = -INFINITY;
+  float m_lane = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < kPerThread; ++j) m = fmaxf(m, v[j]);
-  m = warp_max_f(m);
+  for (int j = 0; j < kPerThread; ++j) m_lane = fmaxf(m_lane, v[j]);
+  // Top-K filter: the K largest lane maxima are K distinct elements of the warp, so an element below
+  // the K-th of them cannot be among the warp's (hence the chunk's) best K, whatever the tie-break.
+  const float tau = warp_kth_bound<K>(m_lane);
+  float m = warp_max_f(m_lane);
   if (lane == 0) s_max[warp] = m;
   __syncthreads();
   m = s_max[0];
@@ -159,10 +177,12 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
   for (int j = 0; j < kPerThread; ++j) {
     const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
-    if (i < n) {
-      sum += exp_nonpos_f64(static_cast<double>(v[j]) - md, s_tab);
-      insert_k<K>(t, Cand{v[j], lo + i});
-    }
+    if (i < n) sum += exp_nonpos_f64(static_cast<double>(v[j]) - md, s_tab);
+  }
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
+    if (i < n && v[j] >= tau) insert_k<K>(t, Cand{v[j], lo + i});
   }
   sum = warp_sum_d(sum);
   warp_merge_k<K>(t, 32);
