@@ -876,6 +876,7 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
 
 }  // namespace attn
 
+static_assert(sizeof(attn::Smem) + 1024 <= 227 * 1024, "shared memory of one CTA (plus alignment slack)");
 size_t attention_smem_bytes() { return sizeof(attn::Smem) + 1024; }
 
 cudaError_t launch_tree_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
