@@ -120,6 +120,8 @@ __global__ void __launch_bounds__(kThreads)
   const int hi = min(vocab, lo + per);
   const float* rows = logits + static_cast<long long>(b) * num_nodes * vocab;
   const bool vec = (vocab % 4) == 0;  // rows then start 16-byte aligned (the base is checked on the host)
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the kernel before this one has completed
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0 && hi > lo) prefetch_l2(rows + lo, hi - lo);  // the root's row, while the tree is read
   // ---- the tree: tokens, parents (validated) and a children list per node
   if (tid == 0) {
@@ -302,20 +304,13 @@ cudaError_t launch_accept(const int32_t* token, const int32_t* parent, const flo
     cudaGetLastError();  // clear a refused attribute / query
     cluster_of[dev].store(cluster, std::memory_order_release);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(batch * cluster);
-  cfg.blockDim = dim3(acc::kThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
   attr.val.clusterDim.x = cluster;
   attr.val.clusterDim.y = 1;
   attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, acc::accept_kernel, token, parent, logits, num_nodes, vocab, max_depth,
-                            accepted_len, path, bonus, status);
+  return launch_pdl(acc::accept_kernel, dim3(batch * cluster), dim3(acc::kThreads), 0, stream, &attr, token, parent,
+                    logits, num_nodes, vocab, max_depth, accepted_len, path, bonus, status);
 }
 
 }  // namespace jf

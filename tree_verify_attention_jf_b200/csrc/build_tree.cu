@@ -139,6 +139,8 @@ __global__ void __launch_bounds__(kThreads)
   const int n = min(kStatsChunk, vocab - lo);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid < 32) s_tab[tid] = g_exp2_frac32[tid];  // visible after the barrier below
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the logits' producer has completed
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   float v[kPerThread];
   if (n == kStatsChunk && (reinterpret_cast<uintptr_t>(x + lo) & 15) == 0) {
     // full, 16-byte aligned chunk: thread t reads float4 number t, t + 256, ...
@@ -380,6 +382,8 @@ __global__ void __launch_bounds__(kExpandThreads)
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid < 32) s.tab[tid] = g_exp2_frac32[tid];
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the row statistics are complete
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __syncthreads();
   // ---- 1. per-depth lse (float64) and top-k: one warp per depth, one lane per chunk partial
   for (int d = 1 + warp; d <= max_depth; d += kExpandThreads / 32) {
@@ -559,16 +563,16 @@ cudaError_t launch_build_tree(const float* logits, const int32_t* root_tokens, i
                               int32_t* depth, RowPartial* partials, int32_t* status, cudaStream_t stream) {
   (void)status;
   const int nchunks = (vocab + kStatsChunk - 1) / kStatsChunk;
-  dim3 g1(nchunks, batch * max_depth);
+  const dim3 g1(nchunks, batch * max_depth), b1(build::kThreads);
+  cudaError_t e;
   if (topk <= 1)
-    build::row_stats_kernel<1><<<g1, build::kThreads, 0, stream>>>(logits, depths, vocab, max_depth, partials);
+    e = launch_pdl(build::row_stats_kernel<1>, g1, b1, 0, stream, nullptr, logits, depths, vocab, max_depth, partials);
   else if (topk <= 2)
-    build::row_stats_kernel<2><<<g1, build::kThreads, 0, stream>>>(logits, depths, vocab, max_depth, partials);
+    e = launch_pdl(build::row_stats_kernel<2>, g1, b1, 0, stream, nullptr, logits, depths, vocab, max_depth, partials);
   else if (topk <= 4)
-    build::row_stats_kernel<4><<<g1, build::kThreads, 0, stream>>>(logits, depths, vocab, max_depth, partials);
+    e = launch_pdl(build::row_stats_kernel<4>, g1, b1, 0, stream, nullptr, logits, depths, vocab, max_depth, partials);
   else
-    build::row_stats_kernel<8><<<g1, build::kThreads, 0, stream>>>(logits, depths, vocab, max_depth, partials);
-  cudaError_t e = cudaGetLastError();
+    e = launch_pdl(build::row_stats_kernel<8>, g1, b1, 0, stream, nullptr, logits, depths, vocab, max_depth, partials);
   if (e != cudaSuccess) return e;
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
@@ -585,20 +589,19 @@ cudaError_t launch_build_tree(const float* logits, const int32_t* root_tokens, i
     }
     attr_set[dev].store(true, std::memory_order_release);
   }
-  const dim3 g2(batch);
+  const dim3 g2(batch), b2(build::kExpandThreads);
+  const RowPartial* part = partials;
   if (topk <= 1)
-    build::expand_kernel<1><<<g2, build::kExpandThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth,
-                                                                        topk, budget, parent, token, score, depth);
-  else if (topk <= 2)
-    build::expand_kernel<2><<<g2, build::kExpandThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth,
-                                                                        topk, budget, parent, token, score, depth);
-  else if (topk <= 4)
-    build::expand_kernel<4><<<g2, build::kExpandThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth,
-                                                                        topk, budget, parent, token, score, depth);
-  else
-    build::expand_kernel<8><<<g2, build::kExpandThreads, dyn, stream>>>(partials, nchunks, root_tokens, max_depth,
-                                                                        topk, budget, parent, token, score, depth);
-  return cudaGetLastError();
+    return launch_pdl(build::expand_kernel<1>, g2, b2, dyn, stream, nullptr, part, nchunks, root_tokens, max_depth,
+                      topk, budget, parent, token, score, depth);
+  if (topk <= 2)
+    return launch_pdl(build::expand_kernel<2>, g2, b2, dyn, stream, nullptr, part, nchunks, root_tokens, max_depth,
+                      topk, budget, parent, token, score, depth);
+  if (topk <= 4)
+    return launch_pdl(build::expand_kernel<4>, g2, b2, dyn, stream, nullptr, part, nchunks, root_tokens, max_depth,
+                      topk, budget, parent, token, score, depth);
+  return launch_pdl(build::expand_kernel<8>, g2, b2, dyn, stream, nullptr, part, nchunks, root_tokens, max_depth,
+                    topk, budget, parent, token, score, depth);
 }
 
 }  // namespace jf

@@ -19,6 +19,30 @@ inline int current_device() {
   return (cudaGetDevice(&d) == cudaSuccess && d >= 0 && d < kMaxDevices) ? d : -1;
 }
 
+// Every kernel of the library is launched with programmatic stream serialisation: it may be scheduled
+// while the kernel before it on the stream is still running, does only local set-up (shared memory,
+// barriers, TMEM, tensor-map prefetches) until its griddepcontrol.wait, and reads or writes global
+// memory only after it.  Each kernel also signals griddepcontrol.launch_dependents early, so the next
+// one's set-up overlaps its tail.  With no kernel before it, the wait returns at once.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              cudaLaunchAttribute* extra, Args&&... args) {
+  cudaLaunchAttribute attrs[2];
+  int n = 0;
+  attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (extra != nullptr) attrs[n++] = *extra;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attrs;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 constexpr int kHeadDim = 128;
 constexpr int kPageSize = 16;
 constexpr int kMaxTreeNodes = 256;          // nodes per sequence in jf_tree_attention

@@ -661,9 +661,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5;
-  // Slot blockIdx.x of the split-unit table is written only by this CTA (if it starts a split unit);
-  // clear what an earlier call left there before anything else.
-  if (tid == 0 && blockIdx.x < kMaxGrid) p.units[blockIdx.x] = make_int4(0, 0, 0, 0);
   // Let the combine kernel be scheduled now; its griddepcontrol.wait still holds it until this grid
   // has finished, but it no longer pays a launch after the last CTA exits.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -702,6 +699,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
+  // the kernel before this one on the stream (which may produce any input) has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // Slot blockIdx.x of the split-unit table is written only by this CTA (if it starts a split unit);
+  // clear what an earlier call left there.
+  if (tid == 0 && blockIdx.x < kMaxGrid) p.units[blockIdx.x] = make_int4(0, 0, 0, 0);
   build_plan(s, p);
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
@@ -775,6 +777,7 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
   __shared__ int4 s_desc[kMaxGrid];
   __shared__ int s_c0[kMaxGrid];
   __shared__ int s_wcount[kCombineThreads / 32];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the attention grid has completed
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // Compact the split units in CTA order (the same list in every block, so that work item i means
@@ -891,21 +894,12 @@ cudaError_t launch_tree_attention(const CUtensorMap& tm_q, const CUtensorMap& tm
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  attn::tree_attention_kernel<<<grid, attn::kThreads, smem, stream>>>(tm_q, tm_k, tm_v, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(attn::tree_attention_kernel, dim3(grid), dim3(attn::kThreads), smem, stream, nullptr,
+                             tm_q, tm_k, tm_v, p);
   if (e != cudaSuccess) return e;
   // The combine kernel may start as soon as the attention grid is scheduled; its griddepcontrol.wait
   // holds it until the attention grid has finished and its writes are visible.
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr.val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * grid);
-  cfg.blockDim = dim3(attn::kCombineThreads);
-  cfg.stream = stream;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn::combine_kernel, p, grid);
+  return launch_pdl(attn::combine_kernel, dim3(2 * grid), dim3(attn::kCombineThreads), 0, stream, nullptr, p, grid);
 }
 
 }  // namespace jf
