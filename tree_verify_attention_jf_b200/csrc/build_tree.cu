@@ -384,6 +384,7 @@ __global__ void __launch_bounds__(kExpandThreads)
   if (tid < 32) s.tab[tid] = g_exp2_frac32[tid];
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the row statistics are complete
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int root_tok = tid == 0 ? root_tokens[b] : 0;  // in flight while the partials are merged
   __syncthreads();
   // ---- 1. per-depth lse (float64) and top-k: one warp per depth, one lane per chunk partial
   for (int d = 1 + warp; d <= max_depth; d += kExpandThreads / 32) {
@@ -420,7 +421,7 @@ __global__ void __launch_bounds__(kExpandThreads)
   int32_t* dep_o = depth_out ? depth_out + static_cast<long long>(b) * budget : nullptr;
   if (tid == 0) {
     par_o[0] = -1;
-    tok_o[0] = root_tokens[b];
+    tok_o[0] = root_tok;
     sc_o[0] = 0.f;
     if (dep_o) dep_o[0] = 0;
     q.lkey[0][0] = 0.0;  // "depth 0": the root

@@ -65,6 +65,7 @@ struct __align__(1024) Smem {
   int meta_ctl;
   int abort_flag;
   int bad_meta;
+  int k_started;  // the K gather has issued its first tile (the V gather's first tile goes after it)
 };
 
 struct Seg {
@@ -239,12 +240,24 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
       const uint32_t mask = __ballot_sync(0xffffffffu, pid >= 0);
       const uint32_t bytes = static_cast<uint32_t>(__popc(mask)) * (kPage * 128u);
       if (!warp_wait(&empty[st], ph ^ 1, abort)) return set_abort(s, p);
+      if (is_v && it == 0) {
+        // The copy engine serves requests in order and the first S needs Q and K only: the kernel's
+        // first V tile is queued behind the first K tile (bounded wait, like every other).
+        const uint64_t t0 = globaltimer();
+        while (*reinterpret_cast<volatile int*>(&s.k_started) == 0) {
+          if (*abort || globaltimer() - t0 > kWaitLimitNs) return set_abort(s, p);
+        }
+      }
       if (lane == 0) mbar_arrive_expect_tx(&full[st], bytes);
       __syncwarp();
       if (pid >= 0) {
         const int half = lane & 1;
         uint8_t* dst = (is_v ? s.v[st] : s.k[st]) + half * kHalfBytes + (lane >> 1) * (kPage * 128);
         tma_load_3d(dst, tm_kv, &full[st], half * 64, g.kvh, pid * kPage);
+      }
+      if (!is_v && it == 0) {
+        __syncwarp();
+        if (lane == 0) *reinterpret_cast<volatile int*>(&s.k_started) = 1;
       }
     }
     ++sidx;
@@ -687,6 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.bar_metaempty[i], kAttnQTiles * kBM);
     }
     s.abort_flag = 0;
+    s.k_started = 0;
     fence_barrier_init();
   }
   if (warp == 0 && (tid & 31) == 0) {
