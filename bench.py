@@ -46,9 +46,9 @@ LAUNCHES_PER_STEP = 5
 # from the captures summarised in profiles/tree_attention_kernel_*.md and profiles/serving_kernels.md), valid
 # only for the kernel source it was taken on: the roofline reports null once that source has changed.
 ATTN_TRAFFIC = {
-    "qwen3_8b": {"bytes": 20.009984e6 + 0.030464e6, "source_sha256": "c67f5208c48f9964917b2e865dab918a35ada932c8750fb2c19c2da8118645ee"},
-    "qwen3_30b_a3b": {"bytes": 2.155419e9 + 0.022077e9, "source_sha256": "c67f5208c48f9964917b2e865dab918a35ada932c8750fb2c19c2da8118645ee"},
-    "serving": {"bytes": 321.87264e6 + 19.57376e6, "source_sha256": "c67f5208c48f9964917b2e865dab918a35ada932c8750fb2c19c2da8118645ee"},
+    "qwen3_8b": {"bytes": 20.016640e6 + 0.028416e6, "source_sha256": "34d20bce1a6b8a6d507cb2485617ff54cc9951fdb81b900ae0c114acae8af2ef"},
+    "qwen3_30b_a3b": {"bytes": 2.143879e9 + 0.021697e9, "source_sha256": "34d20bce1a6b8a6d507cb2485617ff54cc9951fdb81b900ae0c114acae8af2ef"},
+    "serving": {"bytes": 297.490432e6 + 15.588864e6, "source_sha256": "34d20bce1a6b8a6d507cb2485617ff54cc9951fdb81b900ae0c114acae8af2ef"},
 }
 
 
