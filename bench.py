@@ -183,9 +183,10 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------------
 # CPU oracle leg (cpu_baseline and --impl reference)
 # ----------------------------------------------------------------------------------------------
-def oracle_step_rate(cfg, seed, budget_s=15.0, max_steps=40):
-    """Times the oracle over whole steps (build + attention + accept) of the same workload until about
-    `budget_s` seconds of CPU work; returns (nodes/s, steps timed, threads)."""
+def oracle_step_rate(cfg, seed, budget_s=15.0, max_steps=40, warmup=0):
+    """Times the oracle over whole steps (build + attention + accept) of the same workload: `warmup` untimed
+    steps, then steps until about `budget_s` seconds of CPU work or `max_steps` steps; returns (nodes/s, steps
+    timed, seconds, threads)."""
     from oracle.accept import accept as o_accept
     from oracle.build_tree import build_tree as o_build
     from oracle.tree_attention import tree_attention
@@ -199,12 +200,18 @@ def oracle_step_rate(cfg, seed, budget_s=15.0, max_steps=40):
     q = synth.bf16_round(inp["q"])
     tree = o_build(inp["draft"], inp["roots"], cfg["topk"], N, cfg["max_depth"])
     tgt, _ = synth.target_logits_with_path(seed + 2, tree["parent"], tree["token"], cfg["vocab"])
+
+    def one_step():
+        t = o_build(inp["draft"], inp["roots"], cfg["topk"], N, cfg["max_depth"])
+        tree_attention(q, k, v, inp["block_table"], inp["prefix"], inp["offsets"], t["parent"].reshape(-1),
+                       1.0 / np.sqrt(HEAD_DIM), cfg["hkv"])
+        o_accept(t["token"], t["parent"], tgt, cfg["max_depth"])
+
+    for _ in range(warmup):
+        one_step()
     steps, t0 = 0, time.perf_counter()
     while True:
-        tree = o_build(inp["draft"], inp["roots"], cfg["topk"], N, cfg["max_depth"])
-        tree_attention(q, k, v, inp["block_table"], inp["prefix"], inp["offsets"], tree["parent"].reshape(-1),
-                       1.0 / np.sqrt(HEAD_DIM), cfg["hkv"])
-        o_accept(tree["token"], tree["parent"], tgt, cfg["max_depth"])
+        one_step()
         steps += 1
         el = time.perf_counter() - t0
         if el >= budget_s or steps >= max_steps:
@@ -307,10 +314,10 @@ def run_gpu(args, cfg, rank, world, device):
 
     barrier(world)
     torch.cuda.synchronize()
-    sampler = ClockSampler(torch.cuda.get_device_properties(device).uuid, os.path.join(ROOT, "gpurun_out",
-                                                                                        f"clocks_r{rank}.csv")) \
-        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(
-            torch.cuda.get_device_properties(device).uuid, f"/tmp/jf_clocks_r{rank}.csv")
+    import tempfile
+    clocks_dir = args.clocks_dir or tempfile.gettempdir()
+    sampler = ClockSampler(torch.cuda.get_device_properties(device).uuid,
+                           os.path.join(clocks_dir, f"jf_clocks_r{rank}.csv"))
     time.sleep(0.3)
     step_ms = timed(graphs["step"])
     torch.cuda.synchronize()
@@ -370,6 +377,8 @@ def main():
     ap.add_argument("--impl", default="jf", choices=["jf", "reference"])
     ap.add_argument("--workload", default="qwen3_8b", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-dir", default=None, help="where the nvidia-smi clock samples of the timed region go "
+                    "(default: the system temporary directory)")
     args = ap.parse_args()
     cfg = WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", 0))
@@ -388,13 +397,19 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        rate, steps, el, threads = oracle_step_rate(cfg, rank_seed(0))
+        # each step is the oracle over one sequence of the workload (the whole workload when B = 1), so that
+        # the whole --steps K --warmup W run stays within minutes; exactly K steps are timed after W
+        sample_cfg = dict(cfg, batch=1)
+        rate, steps, el, threads = oracle_step_rate(sample_cfg, rank_seed(0), budget_s=float("inf"),
+                                                    max_steps=args.steps, warmup=args.warmup)
+        what = "whole step(s)" if cfg["batch"] == 1 else f"step(s) of one sequence of the {cfg['batch']}"
         line = {"impl": "reference", "metric": metric, "value": rate, "unit": "nodes/s", "n_gpus": args.gpus,
-                "steps": steps, "warmup": 0, "ms_per_step": 1e3 * el / steps, "higher_is_better": True,
+                "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
                 "config": config,
                 "cpu_baseline": {"value": rate, "unit": "nodes/s", "cores": threads, "kind": "oracle",
-                                 "sample": f"{steps} whole step(s) of the workload, {el:.1f} s"},
+                                 "sample": f"{steps} timed {what} (build + attention + accept) after "
+                                           f"{args.warmup} untimed, {el:.1f} s"},
                 "e2e": {"value": rate, "unit": "nodes/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return
