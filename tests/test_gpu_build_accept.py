@@ -55,6 +55,16 @@ def test_build_ties_follow_the_tie_break():
     check_build(x, np.array([3, 4]), 3, 40, 4, margin_guard=False)
 
 
+def test_build_ties_across_chunks():
+    # three logit values over a five-chunk vocabulary: thousands of equal maxima per row, in every lane and
+    # chunk, so the per-warp top-k filter and the (logit desc, id asc) tie-break decide the children; every
+    # depth-1 node ties, so (parent position, rank) orders depth 2.  Depths stay far apart in key.
+    rng = np.random.default_rng(5)
+    x = rng.integers(0, 3, size=(2, 4, 20000)).astype(np.float32)
+    got, ref = check_build(x, np.array([1, 2]), 4, 21, 3, margin_guard=False)
+    assert (got["depth"] == 2).sum() == 2 * 16
+
+
 def gpu_accept(tok, par, tgt, max_depth):
     res = api.accept(torch.from_numpy(np.ascontiguousarray(tok, dtype=np.int32)).cuda(),
                      torch.from_numpy(np.ascontiguousarray(par, dtype=np.int32)).cuda(),

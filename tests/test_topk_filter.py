@@ -1,0 +1,40 @@
+"""Host model of the row-statistics top-K filter: per warp, the bound is the K-th largest distinct lane
+maximum (K rounds of "take the warp max, drop every lane that holds it"), and only elements at or above it
+enter the sorted insertion.  The model checks on random, heavily tied and mostly -inf data that filtering
+never changes the warp's best K by (value desc, id asc)."""
+import numpy as np
+import pytest
+
+
+def kth_bound(lane_max, K):
+    x = lane_max.astype(np.float64).copy()
+    m = -np.inf
+    for _ in range(K):
+        m = x.max()
+        x[x == m] = -np.inf
+    return m
+
+
+def best_k(vals, ids, K):
+    order = sorted(zip((-vals).tolist(), ids.tolist()))
+    return order[:K]
+
+
+@pytest.mark.parametrize("K", [1, 2, 4, 8])
+@pytest.mark.parametrize("kind", ["normal", "ties", "sparse"])
+def test_filter_keeps_the_best_k(K, kind):
+    rng = np.random.default_rng(K * 7 + len(kind))
+    for _ in range(400):
+        if kind == "normal":
+            v = rng.standard_normal((32, 16)).astype(np.float32)
+        elif kind == "ties":
+            v = rng.integers(-2, 2, size=(32, 16)).astype(np.float32)
+        else:
+            v = np.full((32, 16), -np.inf, np.float32)
+            n = int(rng.integers(0, 12))
+            v[rng.integers(0, 32, n), rng.integers(0, 16, n)] = rng.standard_normal(n)
+        # lane l holds elements l * 4 + (j & 3) + 128 * (j // 4) as in the kernel's float4 layout
+        ids = np.array([[(j // 4) * 128 + l * 4 + (j & 3) for j in range(16)] for l in range(32)])
+        tau = kth_bound(v.max(axis=1), K)
+        keep = v >= tau
+        assert best_k(v[keep], ids[keep], K) == best_k(v.ravel(), ids.ravel(), K)
