@@ -180,6 +180,61 @@ class ClockSampler:
         return dict(sm_mhz=statistics.median(sm), sm_max_mhz=max(smax), reasons=sorted(reasons), samples=len(sm))
 
 
+class NvmlSampler:
+    """SM clock and clock-event reasons read through NVML every ~0.2 ms by a background thread, so that a timed
+    region of a few milliseconds still yields samples under load (reads only; no setting is changed).  Falls
+    back to the nvidia-smi sampler when NVML is unavailable."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+
+    def __init__(self, uuid, out_path):
+        import threading
+        self.fallback = None
+        self.sm, self.bits = [], []
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            u = str(uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nv = pynvml
+        except Exception:
+            self.fallback = ClockSampler(uuid, out_path)
+            time.sleep(0.3)  # nvidia-smi's first sample
+            return
+        self.stop_flag = threading.Event()
+        self.running = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+        self.running.wait(timeout=2.0)  # the thread polls before the timed region starts; only later samples count
+        self.sm, self.bits = [], []
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                break
+            self.sm.append(sm)
+            self.bits.append(bits)
+            self.running.set()
+            time.sleep(0.0002)
+
+    def stop(self):
+        if self.fallback is not None:
+            return self.fallback.stop()
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        if not self.sm:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["unsampled"])
+        reasons = sorted({n for b in self.bits for n, m in self.REASONS if b & m})
+        return dict(sm_mhz=statistics.median(self.sm), sm_max_mhz=self.smax, reasons=reasons, samples=len(self.sm),
+                    source="nvml")
+
+
 # ----------------------------------------------------------------------------------------------
 # CPU oracle leg (cpu_baseline and --impl reference)
 # ----------------------------------------------------------------------------------------------
@@ -316,9 +371,8 @@ def run_gpu(args, cfg, rank, world, device):
     torch.cuda.synchronize()
     import tempfile
     clocks_dir = args.clocks_dir or tempfile.gettempdir()
-    sampler = ClockSampler(torch.cuda.get_device_properties(device).uuid,
-                           os.path.join(clocks_dir, f"jf_clocks_r{rank}.csv"))
-    time.sleep(0.3)
+    sampler = NvmlSampler(torch.cuda.get_device_properties(device).uuid,
+                          os.path.join(clocks_dir, f"jf_clocks_r{rank}.csv"))
     step_ms = timed(graphs["step"])
     torch.cuda.synchronize()
     barrier(world)
