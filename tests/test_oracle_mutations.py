@@ -80,3 +80,39 @@ def test_highest_id_tie_break_is_caught(monkeypatch):
         return len(row) - 1 - int(np.argmax(row[::-1]))
     monkeypatch.setattr(acc_mod, "first_argmax", last_argmax)
     assert fails(TA.test_argmax_ties_take_lowest_id)
+
+
+ck_mod = importlib.import_module("oracle.commit_kv")
+from tests import test_oracle_commit as TC
+
+
+def test_commit_ignoring_the_block_table_is_caught(monkeypatch):
+    monkeypatch.setattr(ck_mod, "locate", lambda row, s: (s // 16, s % 16))
+    assert fails(TC.test_hand_worked_example)
+
+
+def test_commit_slots_off_by_one_is_caught(monkeypatch):
+    real = ck_mod.commit_kv
+
+    def off_by_one(k_cache, v_cache, bt, prefix, offs, path, L):
+        return real(k_cache, v_cache, bt, [int(p) - 1 if int(p) > 0 else 0 for p in prefix], offs, path, L)
+    monkeypatch.setattr(TC, "commit_kv", off_by_one)
+    assert fails(TC.test_hand_worked_example)
+
+
+def test_commit_in_place_in_reverse_order_is_caught(monkeypatch):
+    def reverse_in_place(k_cache, v_cache, block_table, prefix_lens, tree_offsets, path, accepted_len):
+        k, v = np.array(k_cache, copy=True), np.array(v_cache, copy=True)
+        newp = np.array(prefix_lens, dtype=np.int64).copy()
+        for b in range(len(prefix_lens)):
+            P, N, L = int(prefix_lens[b]), int(tree_offsets[b + 1]) - int(tree_offsets[b]), int(accepted_len[b])
+            if N == 0:
+                continue
+            for i in range(L, 0, -1):  # no staging, last copy first
+                ps, os_ = ck_mod.locate(block_table[b], P + int(path[b][i]))
+                pd, od = ck_mod.locate(block_table[b], P + i)
+                k[pd, od], v[pd, od] = k[ps, os_].copy(), v[ps, os_].copy()
+            newp[b] = P + L + 1
+        return k, v, newp.astype(np.int32)
+    monkeypatch.setattr(TC, "commit_kv", reverse_in_place)
+    assert fails(TC.test_sources_that_are_later_destinations)
