@@ -334,12 +334,20 @@ def run_gpu(args, cfg, rank, world, device):
         attention()
         accept()
 
+    # the next row after the step: commit the accepted path's K/V into the cache (timed on its own; it rewrites
+    # a few slots of kc/vc in place, which changes no timing)
+    new_prefix = torch.empty_like(prefix)
+
+    def commit():
+        api.commit_kv(kc, vc, bt, prefix, offs, acc_out["path"], acc_out["accepted_len"], new_prefix_lens=new_prefix)
+
     # eager warm-up (loads the library, sets kernel attributes), then one CUDA graph per timed region:
     # the whole step, and each of its three calls alone for the per-kernel times
     step()
     torch.cuda.synchronize()
     graphs = {}
-    for name, fn in (("step", step), ("build_tree", build), ("tree_attention", attention), ("accept", accept)):
+    for name, fn in (("step", step), ("build_tree", build), ("tree_attention", attention), ("accept", accept),
+                     ("commit_kv", commit)):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, capture_error_mode="thread_local"):
             fn()
@@ -380,6 +388,7 @@ def run_gpu(args, cfg, rank, world, device):
     build_ms = timed(graphs["build_tree"])
     attn_ms = timed(graphs["tree_attention"])
     accept_ms = timed(graphs["accept"])
+    commit_ms = timed(graphs["commit_kv"])
     torch.cuda.synchronize()
     del graphs
 
@@ -403,7 +412,8 @@ def run_gpu(args, cfg, rank, world, device):
         e2e_ms.append(e_s.elapsed_time(e_e))
     h2d = draft_h.numel() * 4 + q_h.numel() * 2 + tgt_h.numel() * 4
     d2h = res_h.numel() * 4
-    return dict(step_ms=step_ms, attn_ms=attn_ms, build_ms=build_ms, accept_ms=accept_ms, clocks=clocks,
+    return dict(step_ms=step_ms, attn_ms=attn_ms, build_ms=build_ms, accept_ms=accept_ms, commit_ms=commit_ms,
+                clocks=clocks, accepted=acc_out["accepted_len"].cpu().tolist(),
                 e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, parent=par_h, prefix=inp["prefix"])
 
 
@@ -508,6 +518,10 @@ def main():
         "roofline": roofline(args.workload, tflops, gbs, pk, flops, kv_bytes + qo_bytes + meta_bytes),
         "kernel_ms": {"build_tree": statistics.mean(r["build_ms"]), "tree_attention": attn_ms,
                       "accept": statistics.mean(r["accept_ms"])},
+        # the next row, outside the step: jf_commit_kv of the accepted path (2 * L * Hkv * 256 bytes moved per
+        # sequence, read and written once)
+        "next_rows": {"commit_kv_ms": statistics.mean(r["commit_ms"]), "accepted_len": r["accepted"],
+                      "commit_bytes": sum(2 * 2 * a * cfg["hkv"] * HEAD_DIM * 2 for a in r["accepted"])},
         "time_share": shares,
         "e2e": {"value": job_nodes_per_sec(B, N, world, e2e_step), "unit": "nodes/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},

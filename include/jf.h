@@ -185,6 +185,38 @@ JF_API jf_status jf_accept(const int32_t* token, const int32_t* parent, const fl
                     int batch, int num_nodes, int vocab, int max_depth, int32_t* accepted_len,
                     int32_t* path, int32_t* bonus_token, int32_t* dev_status, jf_stream_t stream);
 
+/* ------------------------------------------------------------------------------------------
+ * jf_commit_kv -- commit the accepted path's K/V into the paged cache, in place.
+ *
+ * The pages run the method inside a paged-KV serving engine [JF section 3] and keep the longest
+ * agreeing prefix of the verified tree [JF section 1]; they leave the cache update itself open.
+ * Reading used: during verification tree node j of sequence b sits at cache slot P + j, with
+ * P = prefix_lens[b] (where jf_tree_attention reads it).  After jf_accept returned path[b] =
+ * [0, n_1, .., n_L] with L = accepted_len[b], slot P + i (i = 1 .. L) receives the K and V of slot
+ * P + n_i (every kv head, all head_dim values), slot P (the root) keeps its own, and
+ * new_prefix_lens[b] = P + L + 1.  Slots from P + L + 1 on are left with unspecified contents.  A
+ * sequence whose tree is empty (tree_offsets[b+1] == tree_offsets[b]) is untouched and keeps P.
+ * Slot s of sequence b is offset s % 16 of page block_table[b, s / 16].
+ *
+ * Layouts: k_cache, v_cache bf16 [num_pages, page_size, num_kv_heads, head_dim], modified in place;
+ *          block_table int32 [batch, max_pages_per_seq]; prefix_lens int32 [batch]; tree_offsets
+ *          int32 [batch+1]; path int32 [batch, max_depth+1] and accepted_len int32 [batch] as
+ *          jf_accept writes them; new_prefix_lens int32 [batch] (it may be prefix_lens itself).
+ * Limits: head_dim == 128, page_size == 16, 1 <= num_kv_heads <= 64, 0 <= max_depth <= 1023,
+ *         num_pages * 16 < 2^31; k_cache and v_cache 16-byte aligned.
+ * Device checks (dev_status = JF_ERR_DEVICE_CHECK; that sequence is left untouched and keeps P):
+ *         accepted_len outside [0, min(max_depth, nodes - 1)], path[0] != 0, a path that does not
+ *         strictly increase or leaves the tree, slots P .. P + nodes - 1 past max_pages_per_seq * 16,
+ *         or one of their page ids outside [0, num_pages).
+ * Ownership: every pointer is caller-owned device memory; nothing is allocated.  Stream-ordered and
+ *         graph-capturable, like the other calls.
+ * ------------------------------------------------------------------------------------------ */
+JF_API jf_status jf_commit_kv(void* k_cache, void* v_cache, const int32_t* block_table, int max_pages_per_seq,
+                       const int32_t* prefix_lens, const int32_t* tree_offsets, const int32_t* path,
+                       const int32_t* accepted_len, int batch, int max_depth, int num_kv_heads, int head_dim,
+                       int page_size, int num_pages, int32_t* new_prefix_lens, int32_t* dev_status,
+                       jf_stream_t stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

@@ -17,7 +17,8 @@ def L():
 def test_exports_every_declared_symbol(L):
     names = _lib.declared_functions()
     assert set(names) == {"jf_status_string", "jf_version", "jf_tree_attention_workspace_size", "jf_tree_attention",
-                          "jf_build_tree_workspace_size", "jf_build_tree", "jf_build_tree_noalloc", "jf_accept"}
+                          "jf_build_tree_workspace_size", "jf_build_tree", "jf_build_tree_noalloc", "jf_accept",
+                          "jf_commit_kv"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -93,3 +94,23 @@ def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         _lib.lib()
+
+
+def test_commit_kv_host_validation(L):
+    def call(**o):
+        a = dict(k=16, v=32, bt=64, maxp=4, pl=128, off=256, path=512, acc=1024, B=2, md=16, hkv=8, d=128, page=16,
+                 pages=64, newp=2048, st=NULL, stream=NULL)
+        a.update(o)
+        return L.jf_commit_kv(a["k"], a["v"], a["bt"], a["maxp"], a["pl"], a["off"], a["path"], a["acc"], a["B"],
+                              a["md"], a["hkv"], a["d"], a["page"], a["pages"], a["newp"], a["st"], a["stream"])
+    assert call(d=64) == _lib.JF_ERR_UNSUPPORTED
+    assert call(page=32) == _lib.JF_ERR_UNSUPPORTED
+    assert call(hkv=65) == _lib.JF_ERR_UNSUPPORTED
+    assert call(md=1024) == _lib.JF_ERR_UNSUPPORTED
+    assert call(hkv=0) == _lib.JF_ERR_INVALID_ARG
+    assert call(B=-1) == _lib.JF_ERR_INVALID_ARG
+    assert call(md=-1) == _lib.JF_ERR_INVALID_ARG
+    assert call(k=NULL) == _lib.JF_ERR_INVALID_ARG
+    assert call(newp=NULL) == _lib.JF_ERR_INVALID_ARG
+    assert call(k=24) == _lib.JF_ERR_INVALID_ARG         # not 16-byte aligned
+    assert call(B=0) == _lib.JF_OK                       # nothing to do, nothing launched

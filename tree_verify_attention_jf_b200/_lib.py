@@ -51,6 +51,8 @@ def lib() -> ctypes.CDLL:
     L.jf_build_tree.restype = i
     L.jf_accept.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp]
     L.jf_accept.restype = i
+    L.jf_commit_kv.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, vp]
+    L.jf_commit_kv.restype = i
     _lib = L
     return L
 

@@ -126,3 +126,33 @@ def accept(token: torch.Tensor, parent: torch.Tensor, target_logits: torch.Tenso
                                 _stream(stream))
     _lib.check("jf_accept", code)
     return out
+
+
+def commit_kv(k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.Tensor, prefix_lens: torch.Tensor,
+              tree_offsets: torch.Tensor, path: torch.Tensor, accepted_len: torch.Tensor,
+              new_prefix_lens: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """jf_commit_kv: moves the accepted path's K/V (path, accepted_len as :func:`accept` returns them) to slots
+    P + 1 .. P + L of each sequence, in place in k_cache / v_cache bf16 [pages, 16, Hkv, 128].  Returns
+    new_prefix_lens int32 [B] (= P + L + 1; it may be prefix_lens itself)."""
+    dev = k_cache.device
+    _need(k_cache, "k_cache", torch.bfloat16, dev)
+    _need(v_cache, "v_cache", torch.bfloat16, dev)
+    for t, name in ((block_table, "block_table"), (prefix_lens, "prefix_lens"), (tree_offsets, "tree_offsets"),
+                    (path, "path"), (accepted_len, "accepted_len")):
+        _need(t, name, torch.int32, dev)
+    if k_cache.shape != v_cache.shape or k_cache.dim() != 4:
+        raise ValueError("k_cache and v_cache must both be [pages, 16, Hkv, 128]")
+    num_pages, page, Hkv, D = k_cache.shape
+    B = prefix_lens.shape[0]
+    if path.dim() != 2 or path.shape[0] != B:
+        raise ValueError("path must be [B, max_depth + 1]")
+    if new_prefix_lens is None:
+        new_prefix_lens = torch.empty(B, dtype=torch.int32, device=dev)
+    _need(new_prefix_lens, "new_prefix_lens", torch.int32, dev)
+    code = _lib.lib().jf_commit_kv(_ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
+                                   _ptr(prefix_lens), _ptr(tree_offsets), _ptr(path), _ptr(accepted_len), B,
+                                   path.shape[1] - 1, Hkv, D, page, num_pages, _ptr(new_prefix_lens), _ptr(dev_status),
+                                   _stream(stream))
+    _lib.check("jf_commit_kv", code)
+    return new_prefix_lens

@@ -195,4 +195,28 @@ jf_status jf_accept(const int32_t* token, const int32_t* parent, const float* ta
   return JF_OK;
 }
 
+jf_status jf_commit_kv(void* k_cache, void* v_cache, const int32_t* block_table, int max_pages_per_seq,
+                       const int32_t* prefix_lens, const int32_t* tree_offsets, const int32_t* path,
+                       const int32_t* accepted_len, int batch, int max_depth, int num_kv_heads, int head_dim,
+                       int page_size, int num_pages, int32_t* new_prefix_lens, int32_t* dev_status,
+                       jf_stream_t stream) {
+  using namespace jf;
+  if (batch < 0 || max_depth < 0 || num_kv_heads <= 0 || max_pages_per_seq <= 0 || num_pages <= 0)
+    return JF_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || page_size != kPageSize || num_kv_heads > kMaxCommitKvHeads ||
+      max_depth >= kMaxAcceptNodes)
+    return JF_ERR_UNSUPPORTED;
+  if (static_cast<long long>(num_pages) * kPageSize >= (1ll << 31)) return JF_ERR_UNSUPPORTED;
+  if (batch == 0) return JF_OK;
+  if (!k_cache || !v_cache || !block_table || !prefix_lens || !tree_offsets || !path || !accepted_len ||
+      !new_prefix_lens)
+    return JF_ERR_INVALID_ARG;
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return JF_ERR_INVALID_ARG;
+  if (launch_commit_kv(k_cache, v_cache, block_table, max_pages_per_seq, prefix_lens, tree_offsets, path,
+                       accepted_len, batch, max_depth, num_kv_heads, num_pages, new_prefix_lens, dev_status,
+                       reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JF_ERR_CUDA;
+  return JF_OK;
+}
+
 }  // extern "C"

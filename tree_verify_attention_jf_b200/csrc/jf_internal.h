@@ -111,4 +111,11 @@ cudaError_t launch_accept(const int32_t* token, const int32_t* parent, const flo
                           int num_nodes, int vocab, int max_depth, int32_t* accepted_len, int32_t* path,
                           int32_t* bonus, int32_t* status, cudaStream_t stream);
 
+// ---- KV commit
+constexpr int kMaxCommitKvHeads = 64;
+cudaError_t launch_commit_kv(void* k_cache, void* v_cache, const int32_t* block_table, int max_pages,
+                             const int32_t* prefix_lens, const int32_t* tree_offsets, const int32_t* path,
+                             const int32_t* accepted_len, int batch, int max_depth, int hkv, int num_pages,
+                             int32_t* new_prefix_lens, int32_t* status, cudaStream_t stream);
+
 }  // namespace jf
