@@ -116,3 +116,34 @@ def test_commit_in_place_in_reverse_order_is_caught(monkeypatch):
         return k, v, newp.astype(np.int32)
     monkeypatch.setattr(TC, "commit_kv", reverse_in_place)
     assert fails(TC.test_sources_that_are_later_destinations)
+
+
+ka_mod = importlib.import_module("oracle.kv_append")
+from tests import test_oracle_kv_append as TK
+
+
+def test_rope_interleaved_pairs_are_caught(monkeypatch):
+    def interleaved(x, pos, theta):
+        x = np.asarray(x, dtype=np.float64)
+        d = x.shape[-1]
+        inv = np.power(float(theta), -2.0 * np.arange(d // 2, dtype=np.float64) / d)
+        ang = np.asarray(pos, dtype=np.float64)[..., None] * inv
+        c, s = np.cos(ang), np.sin(ang)
+        out = x.copy()
+        out[..., 0::2] = x[..., 0::2] * c - x[..., 1::2] * s
+        out[..., 1::2] = x[..., 1::2] * c + x[..., 0::2] * s
+        return out
+    monkeypatch.setattr(TK, "rope", interleaved)
+    assert fails(TK.test_hand_worked_d4)
+
+
+def test_rope_position_off_by_one_is_caught(monkeypatch):
+    orig = ka_mod.node_positions
+    monkeypatch.setattr(ka_mod, "node_positions", lambda p, o, d: orig(p, o, d) - 1)
+    assert fails(TK.test_nodes_land_in_their_slots_with_their_positions)
+
+
+def test_rope_wrong_frequency_base_is_caught(monkeypatch):
+    orig = ka_mod.rope
+    monkeypatch.setattr(TK, "rope", lambda x, pos, theta: orig(x, pos, theta * 10))
+    assert fails(TK.test_matches_complex_formulation, 1e4)
