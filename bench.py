@@ -42,6 +42,7 @@ HEAD_DIM = 128
 PAGE = 16
 L2_FLUSH_BYTES = 256 << 20
 LAUNCHES_PER_STEP = 5
+ROPE_THETA = 1.0e6  # rotary base of the tree K/V append timed beside the step
 # DRAM traffic of one tree_attention_kernel launch per workload (dram__bytes_read.sum + dram__bytes_write.sum
 # from the captures summarised in profiles/tree_attention_kernel_*.md and profiles/serving_kernels.md), valid
 # only for the kernel source it was taken on: the roofline reports null once that source has changed.
@@ -341,13 +342,21 @@ def run_gpu(args, cfg, rank, world, device):
     def commit():
         api.commit_kv(kc, vc, bt, prefix, offs, acc_out["path"], acc_out["accepted_len"], new_prefix_lens=new_prefix)
 
+    # and the row before attention: the tree tokens' K/V (synthetic projections) written into the cache with rotary
+    # positions, q rotated in place (timed on its own)
+    k_new = (torch.randn((B * N, cfg["hkv"], HEAD_DIM), generator=gen, device=device) * 0.5).to(torch.bfloat16)
+    v_new = (torch.randn((B * N, cfg["hkv"], HEAD_DIM), generator=gen, device=device) * 0.5).to(torch.bfloat16)
+
+    def append():
+        api.tree_kv_append(k_new, v_new, kc, vc, bt, prefix, offs, tree["depth"].view(-1), ROPE_THETA, q=q)
+
     # eager warm-up (loads the library, sets kernel attributes), then one CUDA graph per timed region:
     # the whole step, and each of its three calls alone for the per-kernel times
     step()
     torch.cuda.synchronize()
     graphs = {}
     for name, fn in (("step", step), ("build_tree", build), ("tree_attention", attention), ("accept", accept),
-                     ("commit_kv", commit)):
+                     ("commit_kv", commit), ("tree_kv_append", append)):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, capture_error_mode="thread_local"):
             fn()
@@ -389,6 +398,7 @@ def run_gpu(args, cfg, rank, world, device):
     attn_ms = timed(graphs["tree_attention"])
     accept_ms = timed(graphs["accept"])
     commit_ms = timed(graphs["commit_kv"])
+    append_ms = timed(graphs["tree_kv_append"])
     torch.cuda.synchronize()
     del graphs
 
@@ -413,6 +423,7 @@ def run_gpu(args, cfg, rank, world, device):
     h2d = draft_h.numel() * 4 + q_h.numel() * 2 + tgt_h.numel() * 4
     d2h = res_h.numel() * 4
     return dict(step_ms=step_ms, attn_ms=attn_ms, build_ms=build_ms, accept_ms=accept_ms, commit_ms=commit_ms,
+                append_ms=append_ms,
                 clocks=clocks, accepted=acc_out["accepted_len"].cpu().tolist(),
                 e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, parent=par_h, prefix=inp["prefix"])
 
@@ -521,7 +532,10 @@ def main():
         # the next row, outside the step: jf_commit_kv of the accepted path (2 * L * Hkv * 256 bytes moved per
         # sequence, read and written once)
         "next_rows": {"commit_kv_ms": statistics.mean(r["commit_ms"]), "accepted_len": r["accepted"],
-                      "commit_bytes": sum(2 * 2 * a * cfg["hkv"] * HEAD_DIM * 2 for a in r["accepted"])},
+                      "commit_bytes": sum(2 * 2 * a * cfg["hkv"] * HEAD_DIM * 2 for a in r["accepted"]),
+                      # tree K/V append: k_new, v_new read and written, q read and written (bf16)
+                      "tree_kv_append_ms": statistics.mean(r["append_ms"]),
+                      "tree_kv_append_bytes": B * N * (4 * cfg["hkv"] + 2 * cfg["hq"]) * HEAD_DIM * 2},
         "time_share": shares,
         "e2e": {"value": job_nodes_per_sec(B, N, world, e2e_step), "unit": "nodes/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},

@@ -217,6 +217,35 @@ JF_API jf_status jf_commit_kv(void* k_cache, void* v_cache, const int32_t* block
                        int page_size, int num_pages, int32_t* new_prefix_lens, int32_t* dev_status,
                        jf_stream_t stream);
 
+/* ------------------------------------------------------------------------------------------
+ * jf_tree_kv_append -- write the tree tokens' K/V into the paged cache with rotary positions.
+ *
+ * The target verifies the whole tree in one forward pass [JF section 1] inside a paged-KV serving
+ * engine [JF section 3]; the pages leave the cache write and the positions open.  Readings used:
+ * node j of sequence b (flattened index t = tree_offsets[b] + j) goes to cache slot P + j with
+ * P = prefix_lens[b] (where jf_tree_attention reads it); its position is P + depth[t], the root at
+ * depth 0; the rotary embedding turns each pair of head elements (i, i + 64), i < 64, by the angle
+ * pos * rope_theta^(-2i/128), computed in float64 and rounded once to bf16; V is stored unrotated; q,
+ * when not NULL, is rotated in place with the same positions.
+ *
+ * Layouts: k_new, v_new bf16 [total_nodes, num_kv_heads, head_dim]; q bf16 [total_nodes,
+ *          num_q_heads, head_dim] or NULL; k_cache, v_cache bf16 [num_pages, page_size,
+ *          num_kv_heads, head_dim]; block_table int32 [batch, max_pages_per_seq]; prefix_lens int32
+ *          [batch]; tree_offsets int32 [batch+1]; depth int32 [total_nodes] (jf_build_tree's depth
+ *          output, flattened).
+ * Limits: head_dim == 128, page_size == 16, 1 <= batch <= 1024, rope_theta > 0 and finite,
+ *         num_pages * 16 < 2^31; k_new, v_new, q, k_cache, v_cache 16-byte aligned.
+ * Device checks (dev_status = JF_ERR_DEVICE_CHECK; the node is skipped): tree_offsets not starting
+ *         at 0, not ending at total_nodes or decreasing; a negative prefix or depth; a slot past
+ *         max_pages_per_seq * 16; a page id outside [0, num_pages).
+ * Ownership: every pointer is caller-owned device memory; nothing is allocated.
+ * ------------------------------------------------------------------------------------------ */
+JF_API jf_status jf_tree_kv_append(const void* k_new, const void* v_new, void* q, void* k_cache, void* v_cache,
+                            const int32_t* block_table, int max_pages_per_seq, const int32_t* prefix_lens,
+                            const int32_t* tree_offsets, const int32_t* depth, int batch, int total_nodes,
+                            int num_q_heads, int num_kv_heads, int head_dim, int page_size, int num_pages,
+                            float rope_theta, int32_t* dev_status, jf_stream_t stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

@@ -18,7 +18,7 @@ def test_exports_every_declared_symbol(L):
     names = _lib.declared_functions()
     assert set(names) == {"jf_status_string", "jf_version", "jf_tree_attention_workspace_size", "jf_tree_attention",
                           "jf_build_tree_workspace_size", "jf_build_tree", "jf_build_tree_noalloc", "jf_accept",
-                          "jf_commit_kv"}
+                          "jf_commit_kv", "jf_tree_kv_append"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -114,3 +114,24 @@ def test_commit_kv_host_validation(L):
     assert call(newp=NULL) == _lib.JF_ERR_INVALID_ARG
     assert call(k=24) == _lib.JF_ERR_INVALID_ARG         # not 16-byte aligned
     assert call(B=0) == _lib.JF_OK                       # nothing to do, nothing launched
+
+
+def test_tree_kv_append_host_validation(L):
+    def call(**o):
+        a = dict(kn=16, vn=32, q=48, k=64, v=80, bt=96, maxp=4, pl=128, off=256, dep=512, B=2, T=20, hq=32, hkv=8,
+                 d=128, page=16, pages=64, theta=1e6, st=NULL, stream=NULL)
+        a.update(o)
+        return L.jf_tree_kv_append(a["kn"], a["vn"], a["q"], a["k"], a["v"], a["bt"], a["maxp"], a["pl"], a["off"],
+                                   a["dep"], a["B"], a["T"], a["hq"], a["hkv"], a["d"], a["page"], a["pages"],
+                                   a["theta"], a["st"], a["stream"])
+    assert call(d=64) == _lib.JF_ERR_UNSUPPORTED
+    assert call(page=8) == _lib.JF_ERR_UNSUPPORTED
+    assert call(B=2000) == _lib.JF_ERR_UNSUPPORTED
+    assert call(theta=0.0) == _lib.JF_ERR_INVALID_ARG
+    assert call(theta=float("inf")) == _lib.JF_ERR_INVALID_ARG
+    assert call(hkv=0) == _lib.JF_ERR_INVALID_ARG
+    assert call(hq=0) == _lib.JF_ERR_INVALID_ARG             # q given without heads
+    assert call(kn=NULL) == _lib.JF_ERR_INVALID_ARG
+    assert call(q=40) == _lib.JF_ERR_INVALID_ARG             # not 16-byte aligned
+    assert call(T=0) == _lib.JF_OK                           # nothing to do, nothing launched
+    assert call(B=0) == _lib.JF_OK

@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
     L.jf_accept.restype = i
     L.jf_commit_kv.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, vp]
     L.jf_commit_kv.restype = i
+    L.jf_tree_kv_append.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, f, vp, vp]
+    L.jf_tree_kv_append.restype = i
     _lib = L
     return L
 

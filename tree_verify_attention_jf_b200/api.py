@@ -156,3 +156,31 @@ def commit_kv(k_cache: torch.Tensor, v_cache: torch.Tensor, block_table: torch.T
                                    _stream(stream))
     _lib.check("jf_commit_kv", code)
     return new_prefix_lens
+
+
+def tree_kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   block_table: torch.Tensor, prefix_lens: torch.Tensor, tree_offsets: torch.Tensor,
+                   depth: torch.Tensor, rope_theta: float, q: Optional[torch.Tensor] = None,
+                   dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """jf_tree_kv_append: k_new, v_new bf16 [T, Hkv, 128] of the tree tokens go to cache slots P + j of their
+    sequences, K rotated at position P + depth; q bf16 [T, Hq, 128], when given, is rotated in place."""
+    dev = k_cache.device
+    for t, name in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, name, torch.bfloat16, dev)
+    for t, name in ((block_table, "block_table"), (prefix_lens, "prefix_lens"), (tree_offsets, "tree_offsets"),
+                    (depth, "depth")):
+        _need(t, name, torch.int32, dev)
+    if q is not None:
+        _need(q, "q", torch.bfloat16, dev)
+    if k_cache.shape != v_cache.shape or k_cache.dim() != 4 or k_new.shape != v_new.shape or k_new.dim() != 3:
+        raise ValueError("caches must be [pages, 16, Hkv, 128] and k_new / v_new [T, Hkv, 128]")
+    num_pages, page, Hkv, D = k_cache.shape
+    T = k_new.shape[0]
+    if depth.numel() != T or (q is not None and q.shape[0] != T):
+        raise ValueError("depth must have one entry per tree node, q one row per node")
+    B = prefix_lens.shape[0]
+    code = _lib.lib().jf_tree_kv_append(_ptr(k_new), _ptr(v_new), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(block_table), block_table.shape[1], _ptr(prefix_lens), _ptr(tree_offsets),
+                                        _ptr(depth), B, T, q.shape[1] if q is not None else 0, Hkv, D, page, num_pages,
+                                        float(rope_theta), _ptr(dev_status), _stream(stream))
+    _lib.check("jf_tree_kv_append", code)

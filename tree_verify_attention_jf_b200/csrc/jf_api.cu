@@ -219,4 +219,31 @@ jf_status jf_commit_kv(void* k_cache, void* v_cache, const int32_t* block_table,
   return JF_OK;
 }
 
+jf_status jf_tree_kv_append(const void* k_new, const void* v_new, void* q, void* k_cache, void* v_cache,
+                            const int32_t* block_table, int max_pages_per_seq, const int32_t* prefix_lens,
+                            const int32_t* tree_offsets, const int32_t* depth, int batch, int total_nodes,
+                            int num_q_heads, int num_kv_heads, int head_dim, int page_size, int num_pages,
+                            float rope_theta, int32_t* dev_status, jf_stream_t stream) {
+  using namespace jf;
+  if (batch < 0 || total_nodes < 0 || num_kv_heads <= 0 || max_pages_per_seq <= 0 || num_pages <= 0)
+    return JF_ERR_INVALID_ARG;
+  if (q != nullptr && num_q_heads <= 0) return JF_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.f) || !std::isfinite(rope_theta)) return JF_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || page_size != kPageSize) return JF_ERR_UNSUPPORTED;
+  if (batch > kMaxAttnBatch) return JF_ERR_UNSUPPORTED;
+  if (static_cast<long long>(num_pages) * kPageSize >= (1ll << 31)) return JF_ERR_UNSUPPORTED;
+  if (batch == 0 || total_nodes == 0) return JF_OK;
+  if (!k_new || !v_new || !k_cache || !v_cache || !block_table || !prefix_lens || !tree_offsets || !depth)
+    return JF_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      (q != nullptr && !aligned(q, 16)))
+    return JF_ERR_INVALID_ARG;
+  if (launch_tree_kv_append(k_new, v_new, q, k_cache, v_cache, block_table, max_pages_per_seq, prefix_lens,
+                            tree_offsets, depth, batch, total_nodes, q != nullptr ? num_q_heads : 0, num_kv_heads,
+                            num_pages, static_cast<double>(rope_theta), dev_status,
+                            reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JF_ERR_CUDA;
+  return JF_OK;
+}
+
 }  // extern "C"

@@ -118,4 +118,10 @@ cudaError_t launch_commit_kv(void* k_cache, void* v_cache, const int32_t* block_
                              const int32_t* accepted_len, int batch, int max_depth, int hkv, int num_pages,
                              int32_t* new_prefix_lens, int32_t* status, cudaStream_t stream);
 
+// ---- tree K/V append with rotary positions
+cudaError_t launch_tree_kv_append(const void* k_new, const void* v_new, void* q, void* k_cache, void* v_cache,
+                                  const int32_t* block_table, int max_pages, const int32_t* prefix_lens,
+                                  const int32_t* tree_offsets, const int32_t* depth, int batch, int total_nodes,
+                                  int hq, int hkv, int num_pages, double theta, int32_t* status, cudaStream_t stream);
+
 }  // namespace jf
