@@ -147,3 +147,31 @@ def test_rope_wrong_frequency_base_is_caught(monkeypatch):
     orig = ka_mod.rope
     monkeypatch.setattr(TK, "rope", lambda x, pos, theta: orig(x, pos, theta * 10))
     assert fails(TK.test_matches_complex_formulation, 1e4)
+
+
+fp8_mod = importlib.import_module("oracle.fp8_kv")
+from tests import test_oracle_fp8 as TF
+
+
+def test_e4m3_wrong_bias_is_caught(monkeypatch):
+    orig = fp8_mod.e4m3_decode
+    monkeypatch.setattr(TF, "e4m3_decode", lambda c: orig(c) * 2.0)
+    assert fails(TF.test_all_codes_match_torch)
+
+
+def test_e4m3_ties_away_from_zero_is_caught(monkeypatch):
+    def away(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.minimum(np.abs(x), 448.0)
+        vals = fp8_mod._POS
+        idx = np.array([int(np.argmin(np.abs(vals - v) - 1e-12 * (vals > v))) for v in a.ravel()]).reshape(a.shape)
+        return np.where(np.signbit(x), idx | 0x80, idx).astype(np.uint8)
+    monkeypatch.setattr(TF, "e4m3_encode", away)
+    assert fails(TF.test_round_trip_and_ties_to_even)
+
+
+def test_e4m3_no_saturation_is_caught(monkeypatch):
+    orig = fp8_mod.e4m3_encode
+    monkeypatch.setattr(TF, "e4m3_encode", lambda x: np.where(np.abs(np.asarray(x, dtype=np.float64)) > 464.0, 0x7F,
+                                                             orig(x)).astype(np.uint8))
+    assert fails(TF.test_saturation)
