@@ -1,6 +1,5 @@
 """CPU checks of the C ABI: libjf.so loads, exports every function include/jf.h declares, and rejects
 bad arguments on the host before any CUDA call (so these run without a GPU)."""
-import ctypes
 
 import pytest
 

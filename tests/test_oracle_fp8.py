@@ -2,7 +2,6 @@
 float8_e4m3fn conversion (an independent implementation) on all codes and on random values, ties to even,
 saturation, and closed forms of the cache scales in attention."""
 import numpy as np
-import pytest
 import torch
 
 from oracle.fp8_kv import e4m3_decode, e4m3_encode, quantize_cache, tree_attention_fp8

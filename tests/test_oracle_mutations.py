@@ -1,7 +1,6 @@
 """Plants plausible mistakes in the oracle (CPU only, via monkeypatch) and checks that at least one pin
 fails for each, so the pins are known to bite."""
 import numpy as np
-import pytest
 
 import importlib
 

@@ -5,7 +5,6 @@ a CTA that starts segments in mid-range gets correspondingly fewer kv tiles.
 
 Each unit costs SEG_COST + kt positions: SEG_COST leading positions (the price of starting a segment
 in mid-kernel) and then its kt kv tiles."""
-import itertools
 
 import numpy as np
 import pytest
