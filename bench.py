@@ -47,9 +47,9 @@ ROPE_THETA = 1.0e6  # rotary base of the tree K/V append timed beside the step
 # from the captures summarised in profiles/tree_attention_kernel_*.md and profiles/serving_kernels.md), valid
 # only for the kernel source it was taken on: the roofline reports null once that source has changed.
 ATTN_TRAFFIC = {
-    "qwen3_8b": {"bytes": 20.016640e6 + 0.028416e6, "source_sha256": "34d20bce1a6b8a6d507cb2485617ff54cc9951fdb81b900ae0c114acae8af2ef"},
-    "qwen3_30b_a3b": {"bytes": 2.143879e9 + 0.021697e9, "source_sha256": "34d20bce1a6b8a6d507cb2485617ff54cc9951fdb81b900ae0c114acae8af2ef"},
-    "serving": {"bytes": 297.490432e6 + 15.588864e6, "source_sha256": "34d20bce1a6b8a6d507cb2485617ff54cc9951fdb81b900ae0c114acae8af2ef"},
+    "qwen3_8b": {"bytes": 20.016640e6 + 0.028416e6, "source_sha256": "3dbd5be48a438bd65b49f2bc7a6f7075a75070a47c7fa17e665943642079f61d"},
+    "qwen3_30b_a3b": {"bytes": 2.143879e9 + 0.021697e9, "source_sha256": "3dbd5be48a438bd65b49f2bc7a6f7075a75070a47c7fa17e665943642079f61d"},
+    "serving": {"bytes": 297.490432e6 + 15.588864e6, "source_sha256": "3dbd5be48a438bd65b49f2bc7a6f7075a75070a47c7fa17e665943642079f61d"},
 }
 
 

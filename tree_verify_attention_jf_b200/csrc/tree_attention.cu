@@ -16,14 +16,15 @@
 //     (S0 | S1 | O0 | O1) and issues tcgen05.mma: S_i = Q_i K^T (both operands from shared memory,
 //     K-major) and O_i += P_i V with P_i read straight from TMEM (aliasing S_i) and V as an MN-major
 //     shared-memory operand, in the order PV0(j), QK0(j+1), PV1(j), QK1(j+1) so that each softmax
-//     warpgroup works while the tensor core serves the other one.  Warp 3 validates each segment and
-//     builds per-node 256-bit ancestor bitsets by pointer jumping over warp shuffles.  Warps 4-7 and
-//     8-11 (one thread per row of M tile 0 / 1) run the online softmax out of TMEM with a lazy rescale
-//     of O, and the epilogue.
+//     warpgroup works while the tensor core serves the other one.  Warp 3 validates each segment.
+//     Warps 4-7 and 8-11 (one thread per row of M tile 0 / 1) build the per-node 256-bit ancestor
+//     bitsets by pointer jumping in shared memory at each tree-holding segment start, run the online
+//     softmax out of TMEM with a lazy rescale of O, and the epilogue.
 //   * The tree mask only touches tiles that hold tree slots; prefix tiles are unmasked.
 //   * Work split: the flattened (unit, kv tile) space, in which every unit also carries a fixed cost for
-//     the segment start, is cut into equal contiguous ranges, one per CTA (stream-K).  A unit cut between CTAs writes fp32 partials (O, running max, row sum) and its
-//     first CTA records the unit in a descriptor slot; combine_kernel, launched right behind on the
+//     the segment start, is cut into equal contiguous ranges, one per CTA (stream-K).  A unit cut
+//     between CTAs writes fp32 partials (O, running max, row sum) and its first CTA records the unit
+//     in a descriptor slot; combine_kernel, launched right behind on the
 //     same stream with a programmatic dependency, merges each recorded unit's partials and stores the
 //     bf16 output.  Nothing spins on another CTA.
 #include "jf_device.cuh"
