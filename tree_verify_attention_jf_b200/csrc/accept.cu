@@ -8,8 +8,9 @@
 // Design: the walk is a chain of dependent argmaxes over 151936-entry rows, so latency matters more
 // than bandwidth.  Each sequence gets one thread-block cluster (16 CTAs where the GPU allows it,
 // else 8); every CTA reduces its slice of the current row with 16-byte loads issued eight deep, the
-// partial (value, id) pairs are exchanged through distributed shared memory, and every CTA derives
-// the same next node, with one cluster barrier per step.  The children of every node are listed
+// partial (value, id) pairs are exchanged through distributed shared memory (st.async into every
+// CTA's inbox, completing bytes on the receiver's mbarrier; no cluster-wide barrier per step), and
+// every CTA derives the same next node.  The children of every node are listed
 // once at the start; while a row is being reduced, the rows of the current node's children (the
 // only candidates for the next step) are prefetched into L2 with bulk prefetches, so the next step
 // reads from L2.
