@@ -3,11 +3,17 @@
 
 One step = one pass of the whole hot path over one batch: jf_build_tree on the step's draft logits
 (best-first tree of `budget` nodes), jf_tree_attention of every tree node over the paged KV cache
-(prefix + the tree the step just built; Qwen3-8B attention shape by default), jf_accept of the built
-tree against the target logits.  Metric: tree nodes verified per second (whole job), with the
-attention kernel's achieved TFLOP/s and HBM GB/s against the measured B200 peaks.
+(prefix + the tree the step just built), jf_accept of the built tree against the target logits.  The
+default workload is the largest single-GPU one: the Qwen3-30B-A3B attention shape (32 q / 4 kv heads),
+batch 4, 32768-token prefixes, 256-node trees.  Metric: tree nodes verified per second (whole job),
+with the attention kernel's achieved TFLOP/s and HBM GB/s against the measured B200 peaks.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl jf|reference] [--workload qwen3_8b]
+After the step, the same line carries `legs`: the other workloads' calls timed alone -- tree attention
+on the Qwen3-8B shape (256 nodes, 4096 prefix), on the serving batch (16 sequences, 64-node trees,
+prefixes U[1024, 8192]) and on the tiny case (latency), and the tree build and the accept walk at batch
+8 over the full 151936-token vocabulary -- each against its own roofline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl jf|reference] [--workload qwen3_30b_a3b]
 
 N > 1 is launched with torchrun: every rank verifies its own independent batch (weak scaling, no
 collective on the data path); the step time is the max over ranks.  `--impl reference` times the CPU
@@ -41,16 +47,17 @@ WORKLOADS = {
 HEAD_DIM = 128
 PAGE = 16
 L2_FLUSH_BYTES = 256 << 20
+# kernels launched per step: row statistics, best-first expansion, attention, split combine, accept
 LAUNCHES_PER_STEP = 5
 ROPE_THETA = 1.0e6  # rotary base of the tree K/V append timed beside the step
-# DRAM traffic of one tree_attention_kernel launch per workload (dram__bytes_read.sum + dram__bytes_write.sum
-# from the captures summarised in profiles/tree_attention_kernel_*.md and profiles/serving_kernels.md), valid
-# only for the kernel source it was taken on: the roofline reports null once that source has changed.
-ATTN_TRAFFIC = {
-    "qwen3_8b": {"bytes": 20.016640e6 + 0.028416e6, "source_sha256": "3dbd5be48a438bd65b49f2bc7a6f7075a75070a47c7fa17e665943642079f61d"},
-    "qwen3_30b_a3b": {"bytes": 2.143879e9 + 0.021697e9, "source_sha256": "3dbd5be48a438bd65b49f2bc7a6f7075a75070a47c7fa17e665943642079f61d"},
-    "serving": {"bytes": 297.490432e6 + 15.588864e6, "source_sha256": "3dbd5be48a438bd65b49f2bc7a6f7075a75070a47c7fa17e665943642079f61d"},
-}
+DEFAULT_WORKLOAD = "qwen3_30b_a3b"
+# Kernel sources whose hash gates the recorded DRAM traffic below.
+ATTN_SOURCES = ("tree_verify_attention_jf_b200/csrc/tree_attention.cu", "tree_verify_attention_jf_b200/csrc/jf_device.cuh",
+                "tree_verify_attention_jf_b200/csrc/jf_internal.h")
+# DRAM traffic of one tree_attention_kernel launch per workload (dram__bytes_read.sum + dram__bytes_write.sum of an
+# ncu capture of that workload), valid only for the kernel sources it was taken on: the roofline reports null once
+# any of them has changed.  Keys: bench workloads and legs.
+ATTN_TRAFFIC = {}
 
 
 def peaks():
@@ -88,17 +95,22 @@ def make_inputs(cfg, seed):
                 offsets=(np.arange(B + 1) * N).astype(np.int32))
 
 
-def attention_traffic(workload):
-    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary, if the kernel source is
-    still the one that was profiled; else None."""
+def attention_sources_digest():
     import hashlib
+    h = hashlib.sha256()
+    for rel in ATTN_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def attention_traffic(workload):
+    """Per-launch DRAM bytes of the attention kernel recorded from an ncu capture of this workload, if the
+    kernel sources are still the ones that were profiled; else None."""
     rec = ATTN_TRAFFIC.get(workload)
     if rec is None:
         return None
-    src = os.path.join(ROOT, "tree_verify_attention_jf_b200", "csrc", "tree_attention.cu")
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()
-    return rec["bytes"] if digest == rec["source_sha256"] else None
+    return rec["bytes"] if attention_sources_digest() == rec["source_sha256"] else None
 
 
 # Workloads whose attention is bandwidth-bound (arithmetic intensity at or below the ridge) are graded
@@ -137,6 +149,23 @@ def visible_pairs(parent, prefix):
             d[i] = 1 if p < 0 else d[p] + 1
         tot += int(prefix[b]) * parent.shape[1] + int(d.sum())
     return tot
+
+
+def visible_pairs_ragged(parent, offsets, prefix):
+    """visible_pairs for trees of different sizes: parent int [T] local indices, offsets [B+1]."""
+    return sum(visible_pairs(np.asarray(parent[offsets[b]:offsets[b + 1]])[None], [prefix[b]])
+               for b in range(len(prefix)))
+
+
+def attention_work(nodes, hq, hkv, prefix, pairs):
+    """Algorithmic work of one tree-attention call: 4*d flops per visible (query head, key) pair; bytes = the K/V of
+    every sequence's P + N slots read once per kv head, q read and out written once, and the metadata (block
+    table rows in use, parent, prefix length and offsets)."""
+    flops = 4.0 * HEAD_DIM * hq * pairs
+    kv = sum(hkv * (P + n) * HEAD_DIM * 2 * 2 for P, n in zip(prefix, nodes))
+    qo = 2 * sum(nodes) * hq * HEAD_DIM * 2
+    meta = sum(4 * ((P + n + PAGE - 1) // PAGE) + 4 * n + 12 for P, n in zip(prefix, nodes))
+    return flops, kv + qo + meta
 
 
 class ClockSampler:
@@ -283,6 +312,134 @@ def oracle_step_rate(cfg, seed, budget_s=15.0, max_steps=40, warmup=0):
 # ----------------------------------------------------------------------------------------------
 # GPU leg
 # ----------------------------------------------------------------------------------------------
+def graph_timer(args, stream, flush):
+    """Times a callable captured once in a CUDA graph: `steps` replays, each after a 256 MiB write that
+    flushes L2 (outside the events), CUDA events on the launching stream.  Returns the per-replay ms."""
+    import torch
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            fn()
+        return g
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def timed(g, reps=None):
+        for _ in range(3):
+            g.replay()
+        ms = []
+        for _ in range(reps or args.steps):
+            flush.zero_()
+            ev[0].record(stream)
+            g.replay()
+            ev[1].record(stream)
+            ev[1].synchronize()
+            ms.append(ev[0].elapsed_time(ev[1]))
+        return ms
+
+    return capture, timed
+
+
+def attention_leg(name, args, device, capture, timed, pk):
+    """Tree attention alone on one of the seeded attention workloads (the inputs the parity tests use)."""
+    import torch
+
+    from tree_verify_attention_jf_b200 import api, synth, workloads
+
+    inp = workloads.attention_workload(name)
+    bf = lambda a: synth.to_bf16_tensor(a).to(device)
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+    q, kc, vc = bf(inp.q), bf(inp.k_cache), bf(inp.v_cache)
+    bt, pl, offs, par = i32(inp.block_table), i32(inp.prefix_lens), i32(inp.tree_offsets), i32(inp.parent)
+    out = torch.empty_like(q)
+    ws = api.AttentionWorkspace(torch.device(device))
+
+    def call():
+        api.tree_attention(q, kc, vc, bt, pl, offs, par, inp.sm_scale, out=out, workspace=ws)
+
+    call()
+    torch.cuda.synchronize()
+    g = capture(call)
+    ms = statistics.mean(timed(g))
+    del g
+    offs_h = [int(x) for x in inp.tree_offsets]
+    nodes = [offs_h[b + 1] - offs_h[b] for b in range(inp.batch)]
+    prefix = [int(x) for x in inp.prefix_lens]
+    pairs = visible_pairs_ragged(inp.parent, offs_h, prefix)
+    flops, nbytes = attention_work(nodes, inp.num_q_heads, inp.num_kv_heads, prefix, pairs)
+    tflops = flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    leg = {"call": "jf_tree_attention", "ms": ms, "nodes": sum(nodes), "nodes_per_s": sum(nodes) / (ms * 1e-3),
+           "batch": inp.batch, "q_heads": inp.num_q_heads, "kv_heads": inp.num_kv_heads,
+           "prefix": prefix if len(prefix) <= 4 else f"{min(prefix)}..{max(prefix)} (mean {statistics.mean(prefix):.0f})",
+           "algorithmic_flops": flops, "algorithmic_bytes": nbytes, "tflops": tflops, "gbs": gbs,
+           "tensor_frac": tflops / pk["bf16"], "hbm_frac": gbs / pk["hbm"], "traffic": attention_traffic(name)}
+    if name in HBM_BOUND:
+        leg.update(bound="hbm", frac=gbs / pk["hbm"])
+    elif name == "tiny":
+        leg.update(bound="latency", latency_us=ms * 1e3)
+    else:
+        leg.update(bound="tensor", frac=tflops / pk["bf16"])
+    return leg
+
+
+def build_accept_leg(args, device, capture, timed, pk):
+    """Tree build and accept walk at batch 8 over the full vocabulary: draft logits fp32 [8, 16, 151936] with a
+    planted Zipf-peaked head per row, top-4, budget 256, max depth 16; target logits fp32 [8, 256, 151936] that
+    agree with the built tree along a seeded path of length U{1..16}."""
+    import torch
+
+    from tree_verify_attention_jf_b200 import api, synth, workloads
+
+    c = workloads.BUILD
+    B, depths, V, topk, budget, max_depth = (c["batch"], c["depths"], c["vocab"], c["topk"], c["budget"],
+                                             c["max_depth"])
+    x_np, roots_np = workloads.build_inputs()
+    x = torch.from_numpy(x_np).to(device)
+    roots = torch.from_numpy(roots_np).to(device)
+    ws = api.build_tree_workspace(B, depths, V, topk, device)
+    tree = api.build_tree(x, roots, topk, budget, max_depth, workspace=ws)
+    torch.cuda.synchronize()
+    par, tok = tree["parent"].cpu().numpy(), tree["token"].cpu().numpy()
+    tgt_np, paths = synth.target_logits_with_path(workloads.SEEDS["build_accept"] + 100, par, tok, V)
+    tgt = torch.from_numpy(tgt_np).to(device)
+    del tgt_np
+    acc = dict(accepted_len=torch.empty(B, dtype=torch.int32, device=device),
+               path=torch.empty(B, max_depth + 1, dtype=torch.int32, device=device),
+               bonus=torch.empty(B, dtype=torch.int32, device=device))
+
+    def build():
+        api.build_tree(x, roots, topk, budget, max_depth, workspace=ws, out=tree)
+
+    def accept():
+        api.accept(tree["token"], tree["parent"], tgt, max_depth, out=acc)
+
+    build()
+    accept()
+    torch.cuda.synchronize()
+    got = acc["accepted_len"].cpu().tolist()
+    if got != [len(p) - 1 for p in paths]:
+        raise RuntimeError(f"accept leg: accepted lengths {got} != planted {[len(p) - 1 for p in paths]}")
+    gb, ga = capture(build), capture(accept)
+    build_ms = statistics.mean(timed(gb))
+    accept_ms = statistics.mean(timed(ga))
+    del gb, ga
+    build_bytes = B * depths * V * 4
+    accept_bytes = sum((a + 1) * V * 4 for a in got)  # one target row per node on the walk
+    return {
+        "build_tree": {"call": "jf_build_tree", "batch": B, "vocab": V, "depths": depths, "topk": topk,
+                       "budget": budget, "ms": build_ms, "algorithmic_bytes": build_bytes,
+                       "gbs": build_bytes / (build_ms * 1e-3) / 1e9,
+                       "hbm_frac": build_bytes / (build_ms * 1e-3) / 1e9 / pk["hbm"],
+                       "nodes_per_s": B * budget / (build_ms * 1e-3), "bound": "hbm"},
+        "accept": {"call": "jf_accept", "batch": B, "vocab": V, "nodes": budget, "accepted_len": got, "ms": accept_ms,
+                   "algorithmic_bytes": accept_bytes, "gbs": accept_bytes / (accept_ms * 1e-3) / 1e9,
+                   "hbm_frac": accept_bytes / (accept_ms * 1e-3) / 1e9 / pk["hbm"],
+                   "nodes_per_s": B * budget / (accept_ms * 1e-3), "bound": "latency (dependent argmax chain)"},
+    }
+
+
 def run_gpu(args, cfg, rank, world, device):
     import torch
 
@@ -319,6 +476,7 @@ def run_gpu(args, cfg, rank, world, device):
                    bonus=torch.empty(B, dtype=torch.int32, device=device))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
+    capture, timed = graph_timer(args, stream, flush)
 
     def build():
         api.build_tree(draft, roots, cfg["topk"], N, cfg["max_depth"], workspace=ws_build, out=tree)
@@ -354,13 +512,9 @@ def run_gpu(args, cfg, rank, world, device):
     # the whole step, and each of its three calls alone for the per-kernel times
     step()
     torch.cuda.synchronize()
-    graphs = {}
-    for name, fn in (("step", step), ("build_tree", build), ("tree_attention", attention), ("accept", accept),
-                     ("commit_kv", commit), ("tree_kv_append", append)):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, capture_error_mode="thread_local"):
-            fn()
-        graphs[name] = g
+    graphs = {name: capture(fn) for name, fn in (("step", step), ("build_tree", build), ("tree_attention", attention),
+                                                 ("accept", accept), ("commit_kv", commit),
+                                                 ("tree_kv_append", append))}
     for _ in range(args.warmup):
         graphs["step"].replay()
     torch.cuda.synchronize()
@@ -369,31 +523,26 @@ def run_gpu(args, cfg, rank, world, device):
     if got_len != expect_len:
         raise RuntimeError(f"accepted lengths {got_len} != planted {expect_len}")
 
-    # ---- timed region: K graph replays of the whole step, L2 flushed between steps (outside the events);
-    # then K replays of each call alone, for the per-kernel times
+    # ---- timed region: K graph replays of the whole step, L2 flushed between steps (outside the events)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-
-    def timed(g):
-        ms = []
-        for _ in range(args.steps):
-            flush.zero_()
-            ev[0].record(stream)
-            g.replay()
-            ev[1].record(stream)
-            ev[1].synchronize()
-            ms.append(ev[0].elapsed_time(ev[1]))
-        return ms
-
     barrier(world)
     torch.cuda.synchronize()
     import tempfile
     clocks_dir = args.clocks_dir or tempfile.gettempdir()
     sampler = NvmlSampler(torch.cuda.get_device_properties(device).uuid,
                           os.path.join(clocks_dir, f"jf_clocks_r{rank}.csv"))
-    step_ms = timed(graphs["step"])
+    step_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        ev[0].record(stream)
+        graphs["step"].replay()
+        ev[1].record(stream)
+        ev[1].synchronize()
+        step_ms.append(ev[0].elapsed_time(ev[1]))
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop()
+    # then each call alone, for the per-kernel times
     build_ms = timed(graphs["build_tree"])
     attn_ms = timed(graphs["tree_attention"])
     accept_ms = timed(graphs["accept"])
@@ -422,10 +571,24 @@ def run_gpu(args, cfg, rank, world, device):
         e2e_ms.append(e_s.elapsed_time(e_e))
     h2d = draft_h.numel() * 4 + q_h.numel() * 2 + tgt_h.numel() * 4
     d2h = res_h.numel() * 4
-    return dict(step_ms=step_ms, attn_ms=attn_ms, build_ms=build_ms, accept_ms=accept_ms, commit_ms=commit_ms,
-                append_ms=append_ms,
-                clocks=clocks, accepted=acc_out["accepted_len"].cpu().tolist(),
-                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, parent=par_h, prefix=inp["prefix"])
+    r = dict(step_ms=step_ms, attn_ms=attn_ms, build_ms=build_ms, accept_ms=accept_ms, commit_ms=commit_ms,
+             append_ms=append_ms, clocks=clocks, accepted=acc_out["accepted_len"].cpu().tolist(),
+             e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, parent=par_h, prefix=inp["prefix"])
+    del tgt, tgt_h, draft, q, kc, vc, k_new, v_new
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads' calls, each alone (rank 0 of a single-GPU run only)
+    if world == 1 and not args.no_legs:
+        pk = peaks()
+        legs = {}
+        for name in ("qwen3_8b", "serving", "tiny"):
+            if name != args.workload:
+                legs[name] = attention_leg(name, args, device, capture, timed, pk)
+                torch.cuda.empty_cache()
+        legs.update(build_accept_leg(args, device, capture, timed, pk))
+        torch.cuda.empty_cache()
+        r["legs"] = legs
+    return r
 
 
 def barrier(world):
@@ -447,14 +610,17 @@ def max_over_ranks(x, world, device):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="jf", choices=["jf", "reference"])
-    ap.add_argument("--workload", default="qwen3_8b", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-legs", action="store_true", help="skip the other workloads' calls timed after the step")
     ap.add_argument("--clocks-dir", default=None, help="where the nvidia-smi clock samples of the timed region go "
                     "(default: the system temporary directory)")
     args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
     cfg = WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -504,12 +670,9 @@ def main():
     pk = peaks()
     prefixes = [int(x) for x in r["prefix"]]
     pairs = visible_pairs(r["parent"], prefixes)
-    flops = 4.0 * HEAD_DIM * cfg["hq"] * pairs
-    kv_bytes = sum(cfg["hkv"] * (P + N) * HEAD_DIM * 2 * 2 for P in prefixes)
-    qo_bytes = 2 * B * N * cfg["hq"] * HEAD_DIM * 2
-    meta_bytes = sum(4 * ((P + N + PAGE - 1) // PAGE) + 4 * N + 12 for P in prefixes)
+    flops, nbytes = attention_work([N] * B, cfg["hq"], cfg["hkv"], prefixes, pairs)
     tflops = flops / (attn_ms * 1e-3) / 1e12
-    gbs = (kv_bytes + qo_bytes + meta_bytes) / (attn_ms * 1e-3) / 1e9
+    gbs = nbytes / (attn_ms * 1e-3) / 1e9
     shares = {"build_tree": statistics.mean(r["build_ms"]) / mean_step,
               "tree_attention": attn_ms / mean_step, "accept": statistics.mean(r["accept_ms"]) / mean_step}
     if world > 1:
@@ -519,27 +682,30 @@ def main():
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        rate, steps, el, threads = oracle_step_rate(cfg, rank_seed(0))
+        # a bounded sample: whole steps of one sequence of the workload for about 15 s of CPU work
+        sample_cfg = dict(cfg, batch=1)
+        rate, steps, el, threads = oracle_step_rate(sample_cfg, rank_seed(0))
+        what = "whole step(s)" if cfg["batch"] == 1 else f"step(s) of one sequence of the {cfg['batch']}"
         cpu = {"value": rate, "unit": "nodes/s", "cores": threads, "kind": "oracle",
-               "sample": f"{steps} whole step(s) of the same workload (build + attention + accept), {el:.1f} s"}
+               "sample": f"{steps} {what} of the same workload (build + attention + accept), {el:.1f} s"}
     line = {
-        "metric": metric, "value": job_nodes_per_sec(B, N, world, step_ms), "unit": "nodes/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)", "config": config,
-        "roofline": roofline(args.workload, tflops, gbs, pk, flops, kv_bytes + qo_bytes + meta_bytes),
+        "metric": metric, "value": job_nodes_per_sec(B, N, world, step_ms), "unit": "nodes/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)", "config": config,
+        "roofline": roofline(args.workload, tflops, gbs, pk, flops, nbytes),
         "kernel_ms": {"build_tree": statistics.mean(r["build_ms"]), "tree_attention": attn_ms,
                       "accept": statistics.mean(r["accept_ms"])},
-        # the next row, outside the step: jf_commit_kv of the accepted path (2 * L * Hkv * 256 bytes moved per
-        # sequence, read and written once)
+        # the next rows, outside the step: jf_commit_kv of the accepted path (2 * L * Hkv * 256 bytes moved per
+        # sequence, read and written once) and the tree K/V append (k_new, v_new read and written, q read and
+        # written, bf16)
         "next_rows": {"commit_kv_ms": statistics.mean(r["commit_ms"]), "accepted_len": r["accepted"],
                       "commit_bytes": sum(2 * 2 * a * cfg["hkv"] * HEAD_DIM * 2 for a in r["accepted"]),
-                      # tree K/V append: k_new, v_new read and written, q read and written (bf16)
                       "tree_kv_append_ms": statistics.mean(r["append_ms"]),
                       "tree_kv_append_bytes": B * N * (4 * cfg["hkv"] + 2 * cfg["hq"]) * HEAD_DIM * 2},
         "time_share": shares,
+        "legs": r.get("legs"),
         "e2e": {"value": job_nodes_per_sec(B, N, world, e2e_step), "unit": "nodes/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
-        # per step: row statistics + best-first expansion, attention + split combine, accept
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": r["clocks"],
         "cpu_baseline": cpu,

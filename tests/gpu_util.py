@@ -8,6 +8,11 @@ from tree_verify_attention_jf_b200 import api, synth
 MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
 LSE_ABS = 2e-3
+# Error relative to the output's RMS.  The kernel rounds twice in bf16 (unit roundoff u = 2^-9): every softmax
+# weight before the PV product and the output itself; each contributes at most u relative, so the RMS of the
+# error stays below about 2u.  The bound is 4u = 2^-7.  Unlike the absolute bounds it does not loosen when the
+# output is small (long prefixes average V towards zero).
+REL_RMS = 2 ** -7
 
 
 def to_dev(inp: synth.AttentionInputs, device="cuda"):
@@ -41,6 +46,7 @@ def compare(out, ref, lse=None, lse_ref=None, rows=None):
     stats = dict(max_abs=float(err.max()), mean_abs=float(err.mean()), rel_rms=float(np.sqrt(np.mean(err ** 2)) / rms))
     assert stats["max_abs"] <= MAX_ABS, stats
     assert stats["mean_abs"] <= MEAN_ABS, stats
+    assert stats["rel_rms"] <= REL_RMS, stats
     if lse is not None:
         lerr = float(np.abs(lse - lse_ref).max())
         stats["lse_max_abs"] = lerr

@@ -23,8 +23,10 @@ def test_roofline_bound_follows_the_workload():
 
 
 def test_traffic_is_reported_only_for_the_profiled_source(monkeypatch):
-    src = os.path.join(ROOT, "tree_verify_attention_jf_b200", "csrc", "tree_attention.cu")
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    h = hashlib.sha256()
+    for rel in bench.ATTN_SOURCES:
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    digest = h.hexdigest()
     monkeypatch.setattr(bench, "ATTN_TRAFFIC", {"qwen3_8b": {"bytes": 123.0, "source_sha256": digest},
                                                 "serving": {"bytes": 456.0, "source_sha256": "0" * 64}})
     assert bench.attention_traffic("qwen3_8b") == 123.0
@@ -39,6 +41,26 @@ def test_visible_pairs_closed_form():
     assert bench.visible_pairs(parent, [P]) == N * P + N * (N + 1) // 2
     # a star of N roots (parent -1 everywhere): each node sees P + 1
     assert bench.visible_pairs(-np.ones((1, N), np.int64), [P]) == N * (P + 1)
+
+
+def test_ragged_visible_pairs_and_attention_work():
+    # two sequences: a chain of 3 under P = 5, a star of 2 under P = 0
+    parent = np.array([-1, 0, 1, -1, -1])
+    offs, prefix = [0, 3, 5], [5, 0]
+    pairs = bench.visible_pairs_ragged(parent, offs, prefix)
+    assert pairs == (3 * 5 + 1 + 2 + 3) + (0 + 1 + 1)
+    flops, nbytes = bench.attention_work([3, 2], 8, 2, prefix, pairs)
+    assert flops == 4 * 128 * 8 * pairs
+    kv = 2 * (5 + 3) * 128 * 4 + 2 * (0 + 2) * 128 * 4
+    qo = 2 * 5 * 8 * 128 * 2
+    meta = (4 * 1 + 4 * 3 + 12) + (4 * 1 + 4 * 2 + 12)
+    assert nbytes == kv + qo + meta
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    cfg = bench.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    size = lambda c: c["batch"] * c["budget"] * (c["prefix"] if isinstance(c["prefix"], int) else c["prefix"][1])
+    assert all(size(cfg) >= size(c) for c in bench.WORKLOADS.values())
 
 
 def test_job_throughput_counts_every_rank():

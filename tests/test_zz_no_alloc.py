@@ -52,6 +52,8 @@ def test_matches_workspace_variant_on_two_calls_in_a_row():
 
 
 def test_rejects_calls_beyond_the_scratch_limit():
-    # 64 sequences x 16 depths x 38 chunks x 80 bytes > 1 MiB: refused before anything is launched
-    code = noalloc_fn()(16, 32, 64, 16, 151936, 4, 256, 16, 64, 128, 256, None, None, None)
+    # 64 sequences x 16 depths x 38 chunks x 80 bytes > 1 MiB: refused before anything is launched.  Every
+    # pointer is null, so that if the size check ever stopped refusing this call, the null-pointer check
+    # would still turn it into JF_ERR_INVALID_ARG (and this test would fail) without launching a kernel.
+    code = noalloc_fn()(None, None, 64, 16, 151936, 4, 256, 16, None, None, None, None, None, None)
     assert code == _lib.JF_ERR_UNSUPPORTED

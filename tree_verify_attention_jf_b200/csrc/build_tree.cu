@@ -614,6 +614,7 @@ cudaError_t launch_build_tree(const float* logits, const int32_t* root_tokens, i
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB, held by every GPU that loads the library
+static_assert(sizeof(jf::RowPartial) == 80, "the documented limit of jf_build_tree_noalloc counts 80 B per row partial");
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_noalloc_mutex;

@@ -44,8 +44,8 @@ constexpr int kTileBytes = 2 * kHalfBytes;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmS = 0;    // S_i at column 128 * i
 constexpr uint32_t kTmO = 256;  // O_i at column 256 + 128 * i
-constexpr float kRescaleThreshold = 8.0f;
-constexpr int kSegCost = 3;  // kv tiles' worth of time that starting a segment in mid-kernel costs  // log2 units: P may grow up to 2^8 before O is rescaled
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow up to 2^8 before O is rescaled
+constexpr int kSegCost = 3;  // kv tiles' worth of time that starting a segment in mid-kernel costs
 
 struct __align__(1024) Smem {
   uint8_t q[kAttnQTiles][kTileBytes];
