@@ -5,7 +5,8 @@ define: tree-causal attention over a paged KV cache (``tree_attention``), best-f
 construction by cumulative draft log-probability under a budget (``build_tree``), the greedy
 acceptance walk (``accept``), the commit of the accepted path's K/V into the cache
 (``commit_kv``), the write of the tree tokens' rotated K/V into the cache (``tree_kv_append``),
-and tree attention over an 8-bit E4M3 cache (``tree_attention_fp8``; no kernel yet).  It shares no code with the CUDA library and never imports it.
+tree attention over an 8-bit E4M3 cache (``tree_attention_fp8``), and the round-by-round best-first
+expansion from per-node (path-conditioned) draft logits (``expand_frontier``, ``grow_tree``).  It shares no code with the CUDA library and never imports it.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference`` legs of
 ``bench.py`` may import this package.  The product path (the ``libjf.so`` C-ABI and its Python
@@ -25,3 +26,4 @@ from .accept import accept  # noqa: F401
 from .commit_kv import commit_kv  # noqa: F401
 from .kv_append import rope, tree_kv_append  # noqa: F401
 from .fp8_kv import e4m3_decode, e4m3_encode, quantize_cache, tree_attention_fp8  # noqa: F401
+from .frontier import FrontierState, expand_frontier, grow_tree, start_tree  # noqa: F401

@@ -7,7 +7,9 @@ import importlib
 acc_mod = importlib.import_module("oracle.accept")
 bt_mod = importlib.import_module("oracle.build_tree")
 ta_mod = importlib.import_module("oracle.tree_attention")
+fr_mod = importlib.import_module("oracle.frontier")
 from tests import test_oracle_accept as TA
+from tests import test_oracle_frontier as TFR
 from tests import test_oracle_attention as TT
 from tests import test_oracle_build as TB
 
@@ -174,3 +176,42 @@ def test_e4m3_no_saturation_is_caught(monkeypatch):
     monkeypatch.setattr(TF, "e4m3_encode", lambda x: np.where(np.abs(np.asarray(x, dtype=np.float64)) > 464.0, 0x7F,
                                                              orig(x)).astype(np.uint8))
     assert fails(TF.test_saturation)
+
+
+def test_frontier_key_without_the_parent_score_is_caught(monkeypatch):
+    monkeypatch.setattr(fr_mod, "candidate_key", lambda parent_key, lp: lp)
+    assert fails(TFR.test_width_one_with_path_conditioned_rows_is_exact_best_first, 11, 2, 4, 20)
+
+
+def test_frontier_reoffering_taken_children_is_caught(monkeypatch):
+    monkeypatch.setattr(fr_mod, "untaken", lambda state, u: range(len(state.cand_tok[u])))
+    assert fails(TFR.test_invariants, 7)
+
+
+def test_frontier_lp_without_the_normaliser_is_caught(monkeypatch):
+    def children_no_lse(row, topk):
+        row = np.asarray(row)
+        tok = fr_mod.topk_tokens(row, topk)
+        return tok, row[tok].astype(np.float64)
+    monkeypatch.setattr(fr_mod, "node_children", children_no_lse)
+    assert fails(TFR.test_invariants, 3)
+
+
+def test_frontier_children_of_this_rounds_picks_are_caught(monkeypatch):
+    # a round that scores every node it adds at once (as if its row were already known) loses the round structure:
+    # children join in the same round as their parent
+    orig = fr_mod.expand_frontier
+
+    def eager(state, rows, root_token, topk, max_depth, width):
+        added = orig(state, rows, root_token, topk, max_depth, 1)
+        while added < width and state.num_nodes < state.budget:
+            fr_mod.start_tree(state, root_token)
+            new = list(state.frontier())
+            extra = [TFR.synth.path_logits(31 + width, state.path_tokens(i), 500) for i in new]
+            a = orig(state, extra, root_token, topk, max_depth, 1)
+            if a == 0:
+                break
+            added += a
+        return added
+    monkeypatch.setattr(fr_mod, "expand_frontier", eager)
+    assert fails(TFR.test_invariants, 7)

@@ -194,6 +194,23 @@ def draft_logits(seed: int, batch: int, depths: int, vocab: int, sigma: float = 
     return x, roots
 
 
+def path_logits(seed: int, path: tuple, vocab: int, sigma: float = 2.0, plant: int = 8) -> np.ndarray:
+    """Draft logits fp32 [vocab] at one tree node, drawn from a generator seeded by ``seed`` and the node's root
+    path (its token ids, root first), so that the same path always gets the same row: the stand-in for a draft
+    head whose output at a node depends on that node's path.  Same recipe as :func:`draft_logits` rows:
+    N(0, sigma^2) with ``plant`` distinct ids lifted to rowmax + c - s*ln(r), c ~ U(4, 10), s ~ U(0.8, 1.5)."""
+    rng = np.random.default_rng(np.random.SeedSequence([int(seed), len(path)] + [int(t) for t in path]))
+    x = rng.standard_normal(vocab, dtype=np.float32) * np.float32(sigma)
+    if plant:
+        toks = rng.choice(vocab, size=min(plant, vocab), replace=False)
+        c = rng.uniform(4.0, 10.0)
+        s = rng.uniform(0.8, 1.5)
+        top = float(x.max())
+        for r, t in enumerate(toks, start=1):
+            x[t] = np.float32(top + c - s * np.log(r))
+    return x
+
+
 def target_logits_with_path(seed: int, parent: np.ndarray, token: np.ndarray, vocab: int,
                             path_len: Optional[list[int]] = None, sigma: float = 2.0,
                             lift: float = 4.0) -> tuple[np.ndarray, list[list[int]]]:
