@@ -165,6 +165,54 @@ JF_API jf_status jf_build_tree_noalloc(const float* draft_logits, const int32_t*
                                        int32_t* dev_status, jf_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * jf_expand_frontier -- one round of best-first tree construction from per-node draft logits.
+ *
+ * Defines [JF section 2: the draft head conditions every node on its own root path, the branch
+ * factorisation q(pi(v)|x) = prod_{u in pi(v)} q(y_u | x, h, pi_<u); the tree is built best-first by
+ * cumulative draft log-probability up to a budget].  With path-conditioned logits a node's children can
+ * be scored only after the draft head has run on that node, so the tree grows in rounds; each call is
+ * one round.  At entry, sequence b's tree holds num_nodes[b] nodes and its frontier is the nodes
+ * [frontier_begin[b], num_nodes[b]); row j of node_logits[b] is the draft head's next-token logits at
+ * frontier node frontier_begin[b] + j.  num_nodes[b] == 0 starts a new tree: node 0 = root_tokens[b]
+ * (parent -1, depth 0, score 0) is created and is the whole frontier, scored by row 0.  Steps:
+ *   1. every frontier node u below max_depth gets its candidate children: the top-k tokens of its
+ *      row by (logit descending, token id ascending), with lp = x_tok - lse (float64 lse and exp,
+ *      as jf_build_tree);
+ *   2. among the untaken candidates (u, r) of every node scored so far, keyed key(u) + lp_u[r] in
+ *      float64, the best min(width, budget - num_nodes[b]) by (key descending, depth ascending,
+ *      parent index ascending, rank ascending) are appended in that order (score = key rounded to
+ *      fp32);
+ *   3. frontier_begin[b] = the old num_nodes[b]; num_nodes[b] grows by the nodes appended (fewer
+ *      than width only at the budget or when no candidate is left), which form the next frontier.
+ * With width 1 the rounds reproduce jf_build_tree's pop order when every node's row is its depth's
+ * row.  Rows past a sequence's frontier are never read; a sequence whose tree already holds `budget`
+ * nodes is left as it is and none of its rows is read.
+ *
+ * Layouts: node_logits fp32 [batch, frontier_rows, vocab]; root_tokens int32 [batch];
+ *          parent, token, depth int32 [batch, budget] and score fp32 [batch, budget], in/out (the
+ *          tree so far; entries past num_nodes[b] are unspecified); num_nodes, frontier_begin int32
+ *          [batch], in/out.
+ * state: jf_expand_frontier_state_size(batch, budget, topk) bytes, caller-owned, carried between
+ *        the rounds of one tree (each node's float64 key and its candidates); it needs no
+ *        initialisation before a tree's first round and must not be modified between rounds.
+ * workspace: jf_expand_frontier_workspace_size(batch, frontier_rows, vocab) bytes, reusable.
+ * Limits: 1 <= topk <= 8, topk <= vocab, 1 <= budget <= 256, 1 <= max_depth, 1 <= width,
+ *         1 <= frontier_rows <= 256, batch * frontier_rows <= 65535.
+ * Device checks (JF_ERR_DEVICE_CHECK, sequence left unchanged): num_nodes[b] outside [0, budget],
+ * frontier_begin[b] outside [0, num_nodes[b]], or a frontier longer than frontier_rows.
+ * ------------------------------------------------------------------------------------------ */
+JF_API size_t jf_expand_frontier_state_size(int batch, int budget, int topk);
+
+JF_API size_t jf_expand_frontier_workspace_size(int batch, int frontier_rows, int vocab);
+
+JF_API jf_status jf_expand_frontier(const float* node_logits, const int32_t* root_tokens, int batch,
+                                    int frontier_rows, int vocab, int topk, int budget, int max_depth,
+                                    int width, int32_t* parent, int32_t* token, float* score,
+                                    int32_t* depth, int32_t* num_nodes, int32_t* frontier_begin,
+                                    void* state, size_t state_bytes, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status, jf_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * jf_accept -- greedy acceptance walk over the verified tree.
  *
  * Defines [JF section 1: the target verifies the drafted tokens in parallel and keeps the longest

@@ -17,7 +17,8 @@ def test_exports_every_declared_symbol(L):
     names = _lib.declared_functions()
     assert set(names) == {"jf_status_string", "jf_version", "jf_tree_attention_workspace_size", "jf_tree_attention",
                           "jf_build_tree_workspace_size", "jf_build_tree", "jf_build_tree_noalloc", "jf_accept",
-                          "jf_commit_kv", "jf_tree_kv_append"}
+                          "jf_commit_kv", "jf_tree_kv_append", "jf_expand_frontier_state_size",
+                          "jf_expand_frontier_workspace_size", "jf_expand_frontier"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -134,3 +135,25 @@ def test_tree_kv_append_host_validation(L):
     assert call(q=40) == _lib.JF_ERR_INVALID_ARG             # not 16-byte aligned
     assert call(T=0) == _lib.JF_OK                           # nothing to do, nothing launched
     assert call(B=0) == _lib.JF_OK
+
+
+def test_expand_frontier_host_validation(L):
+    # every pointer is null: a call that passed the size checks would stop at the null-pointer check
+    def call(**over):
+        a = dict(batch=2, rows=4, V=1000, topk=4, budget=64, max_depth=8, width=16)
+        a.update(over)
+        return L.jf_expand_frontier(None, None, a["batch"], a["rows"], a["V"], a["topk"], a["budget"],
+                                    a["max_depth"], a["width"], None, None, None, None, None, None, None, 0, None, 0,
+                                    None, None)
+    assert call() == _lib.JF_ERR_INVALID_ARG  # null pointers
+    assert call(batch=0) == _lib.JF_OK
+    assert call(topk=9) == _lib.JF_ERR_UNSUPPORTED
+    assert call(budget=257) == _lib.JF_ERR_UNSUPPORTED
+    assert call(rows=257) == _lib.JF_ERR_UNSUPPORTED
+    assert call(batch=300, rows=256) == _lib.JF_ERR_UNSUPPORTED  # grid rows > 65535
+    assert call(topk=5, V=4) == _lib.JF_ERR_INVALID_ARG
+    for bad in (dict(width=0), dict(max_depth=0), dict(rows=0), dict(budget=0), dict(topk=0), dict(V=0),
+                dict(batch=-1)):
+        assert call(**bad) == _lib.JF_ERR_INVALID_ARG, bad
+    assert L.jf_expand_frontier_state_size(2, 64, 4) >= 2 * 64 * (8 + 4 * 8 + 4 * 4 + 4)
+    assert L.jf_expand_frontier_workspace_size(2, 4, 4096) == 2 * 4 * 1 * 80

@@ -49,6 +49,12 @@ def lib() -> ctypes.CDLL:
     L.jf_build_tree_workspace_size.restype = sz
     L.jf_build_tree.argtypes = [vp, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, sz, vp, vp]
     L.jf_build_tree.restype = i
+    L.jf_expand_frontier_state_size.argtypes = [i, i, i]
+    L.jf_expand_frontier_state_size.restype = sz
+    L.jf_expand_frontier_workspace_size.argtypes = [i, i, i]
+    L.jf_expand_frontier_workspace_size.restype = sz
+    L.jf_expand_frontier.argtypes = [vp, vp, i, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, sz, vp, sz, vp, vp]
+    L.jf_expand_frontier.restype = i
     L.jf_accept.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp]
     L.jf_accept.restype = i
     L.jf_commit_kv.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, vp]

@@ -108,6 +108,53 @@ def build_tree(draft_logits: torch.Tensor, root_tokens: torch.Tensor, topk: int,
     return out
 
 
+class FrontierTree:
+    """A batch of trees grown round by round with :func:`expand_frontier`: the tree arrays (parent, token, depth
+    int32 [B, budget], score fp32 [B, budget]), the node counts and frontier starts (int32 [B]) and the state the
+    library carries between rounds.  ``reset()`` starts new trees (the next round creates the roots)."""
+
+    def __init__(self, batch: int, budget: int, topk: int, device):
+        self.batch, self.budget, self.topk = batch, budget, topk
+        self.parent = torch.full((batch, budget), -1, dtype=torch.int32, device=device)
+        self.token = torch.zeros(batch, budget, dtype=torch.int32, device=device)
+        self.depth = torch.zeros(batch, budget, dtype=torch.int32, device=device)
+        self.score = torch.zeros(batch, budget, dtype=torch.float32, device=device)
+        self.num_nodes = torch.zeros(batch, dtype=torch.int32, device=device)
+        self.frontier_begin = torch.zeros(batch, dtype=torch.int32, device=device)
+        n = _lib.lib().jf_expand_frontier_state_size(batch, budget, topk)
+        self.state = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+    def reset(self) -> None:
+        self.num_nodes.zero_()
+        self.frontier_begin.zero_()
+
+
+def expand_frontier_workspace(batch: int, frontier_rows: int, vocab: int, device) -> torch.Tensor:
+    n = _lib.lib().jf_expand_frontier_workspace_size(batch, frontier_rows, vocab)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def expand_frontier(node_logits: torch.Tensor, root_tokens: torch.Tensor, tree: FrontierTree, max_depth: int,
+                    width: int, workspace: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+                    stream=None) -> FrontierTree:
+    """jf_expand_frontier: one round.  node_logits fp32 [B, F, V] (row j of sequence b = the draft head's logits at
+    node tree.frontier_begin[b] + j); root_tokens int32 [B].  Updates ``tree`` in place and returns it."""
+    dev = node_logits.device
+    B, F, V = node_logits.shape
+    _need(node_logits, "node_logits", torch.float32, dev)
+    _need(root_tokens, "root_tokens", torch.int32, dev)
+    if B != tree.batch:
+        raise ValueError("node_logits and tree have different batch sizes")
+    if workspace is None:
+        workspace = expand_frontier_workspace(B, F, V, dev)
+    code = _lib.lib().jf_expand_frontier(
+        _ptr(node_logits), _ptr(root_tokens), B, F, V, tree.topk, tree.budget, max_depth, width, _ptr(tree.parent),
+        _ptr(tree.token), _ptr(tree.score), _ptr(tree.depth), _ptr(tree.num_nodes), _ptr(tree.frontier_begin),
+        _ptr(tree.state), tree.state.numel(), _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream))
+    _lib.check("jf_expand_frontier", code)
+    return tree
+
+
 def accept(token: torch.Tensor, parent: torch.Tensor, target_logits: torch.Tensor, max_depth: int,
            out: Optional[dict] = None, dev_status: Optional[torch.Tensor] = None, stream=None) -> dict:
     """jf_accept: token, parent int32 [B, N]; target_logits fp32 [B, N, V] -> dict of accepted_len int32 [B],

@@ -12,7 +12,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libjf.so")
-SOURCES = ["jf_api.cu", "tree_attention.cu", "build_tree.cu", "accept.cu", "commit_kv.cu", "kv_append.cu"]
+SOURCES = ["jf_api.cu", "tree_attention.cu", "build_tree.cu", "frontier.cu", "accept.cu", "commit_kv.cu",
+           "kv_append.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

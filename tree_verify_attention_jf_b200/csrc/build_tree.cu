@@ -23,111 +23,24 @@
 #include "jf_device.cuh"
 #include "jf_internal.h"
 #include "jf_math.cuh"
+#include "build_common.cuh"
 
 namespace jf {
 namespace build {
-
-__device__ const double g_exp2_frac32[32] = JF_EXP2_FRAC32;
-
-constexpr int kThreads = 256;
-constexpr int kPerThread = kStatsChunk / kThreads;  // 16
-constexpr int kSlots = kMaxDepths * kMaxTopk / 32;  // queue slots per lane (16)
-
-struct Cand {
-  float v;
-  int id;
-};
-
-__device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
-  return a.v > b.v || (a.v == b.v && a.id < b.id);
-}
-
-__device__ __forceinline__ void cswap(Cand& a, Cand& b) {  // after: a better-or-equal than b
-  if (better(b, a)) {
-    const Cand t = a;
-    a = b;
-    b = t;
-  }
-}
-
-// keep t[] sorted best-first; insert x if it beats the last entry
-template <int K>
-__device__ __forceinline__ void insert_k(Cand (&t)[K], Cand x) {
-  if (!better(x, t[K - 1])) return;
-  t[K - 1] = x;
-#pragma unroll
-  for (int i = K - 1; i > 0; --i) cswap(t[i - 1], t[i]);
-}
-
-// t := best K of t U u (both sorted best-first), via a bitonic merge (K a power of two)
-template <int K>
-__device__ __forceinline__ void merge_k(Cand (&t)[K], const Cand (&u)[K]) {
-#pragma unroll
-  for (int i = 0; i < K; ++i) {
-    const Cand o = u[K - 1 - i];
-    if (better(o, t[i])) t[i] = o;
-  }
-  // t is now bitonic; sort it best-first
-#pragma unroll
-  for (int span = K / 2; span > 0; span >>= 1) {
-#pragma unroll
-    for (int i = 0; i < K; ++i) {
-      if ((i & span) == 0) cswap(t[i], t[i + span]);
-    }
-  }
-}
-
-template <int K>
-__device__ __forceinline__ void warp_merge_k(Cand (&t)[K], int width) {
-  for (int off = width / 2; off > 0; off >>= 1) {
-    Cand u[K];
-#pragma unroll
-    for (int i = 0; i < K; ++i) {
-      u[i].v = __shfl_xor_sync(0xffffffffu, t[i].v, off);
-      u[i].id = __shfl_xor_sync(0xffffffffu, t[i].id, off);
-    }
-    merge_k<K>(t, u);
-  }
-}
-
-__device__ __forceinline__ void merge8(Cand (&t)[kMaxTopk], const Cand (&u)[kMaxTopk]) { merge_k<kMaxTopk>(t, u); }
-__device__ __forceinline__ void warp_merge8(Cand (&t)[kMaxTopk], int width) { warp_merge_k<kMaxTopk>(t, width); }
-
-__device__ __forceinline__ double warp_sum_d(double x) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-  return x;
-}
-
-__device__ __forceinline__ float warp_max_f(float x) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
-  return x;
-}
-
-// A lower bound on the K-th largest of the warp's 32 values: K rounds of "take the warp max, drop every
-// lane that holds it".  Ties are dropped together, so the result is the K-th largest distinct value
-// (or -inf if there are fewer), which never exceeds the K-th largest counted with multiplicity.
-template <int K>
-__device__ __forceinline__ float warp_kth_bound(float x) {
-  float m = -INFINITY;
-#pragma unroll
-  for (int r = 0; r < K; ++r) {
-    m = warp_max_f(x);
-    if (x == m) x = -INFINITY;
-  }
-  return m;
-}
 
 // ------------------------------------------------------------------------------------------------
 // Kernel 1: chunk statistics.  grid = (chunks, batch * max_depth)
 // ------------------------------------------------------------------------------------------------
 // K: the per-chunk list length, the smallest power of two >= topk (only the best topk of a row can
 // ever become children, so shorter lists are exact and much cheaper to maintain).
+// With lim_nodes / lim_begin (the frontier expansion), row (b, d) is read only if d is below sequence b's frontier
+// size: lim_nodes[b] - lim_begin[b] rows, 1 (the root's) for a tree that has no node yet, none for a tree that
+// already holds lim_budget nodes.
 template <int K>
 __global__ void __launch_bounds__(kThreads)
     row_stats_kernel(const float* __restrict__ logits, int depths, int vocab, int max_depth,
-                     RowPartial* __restrict__ out) {
+                     RowPartial* __restrict__ out, const int32_t* __restrict__ lim_nodes,
+                     const int32_t* __restrict__ lim_begin, int lim_budget) {
   __shared__ float s_max[kThreads / 32];
   __shared__ double s_sum[kThreads / 32];
   __shared__ Cand s_top[kThreads / 32][K];
@@ -141,6 +54,11 @@ __global__ void __launch_bounds__(kThreads)
   if (tid < 32) s_tab[tid] = g_exp2_frac32[tid];  // visible after the barrier below
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the logits' producer has completed
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (lim_nodes != nullptr) {
+    const int n = lim_nodes[b];
+    const int rows = (n == 0) ? 1 : (n >= lim_budget ? 0 : n - lim_begin[b]);
+    if (d >= rows) return;  // uniform over the CTA: a row outside the frontier is never read
+  }
   float v[kPerThread];
   if (n == kStatsChunk && (reinterpret_cast<uintptr_t>(x + lo) & 15) == 0) {
     // full, 16-byte aligned chunk: thread t reads float4 number t, t + 256, ...
@@ -217,18 +135,6 @@ __global__ void __launch_bounds__(kThreads)
 // ------------------------------------------------------------------------------------------------
 // Kernel 2: merge + best-first expansion.  grid = batch, block = 256
 // ------------------------------------------------------------------------------------------------
-// Order-preserving map of a (non-NaN) double to an unsigned integer: a < b as doubles iff
-// ord_key(a) < ord_key(b).  -0 is taken as +0 so that equal doubles give equal keys.
-__device__ __forceinline__ unsigned long long ord_key(double k) {
-  if (k == 0.0) k = 0.0;
-  const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(k));
-  return (bits >> 63) ? ~bits : (bits | 0x8000000000000000ull);
-}
-__device__ __forceinline__ double key_of_ord(unsigned long long o) {
-  const unsigned long long bits = (o >> 63) ? (o & 0x7fffffffffffffffull) : ~o;
-  return __longlong_as_double(static_cast<long long>(bits));
-}
-
 struct ExpandSmem {
   double tab[32];                       // 2^(j/32) for exp_nonpos_f64
   double lp[kMaxDepths + 1][kMaxTopk];  // lp[d][r], d = 1..max_depth
@@ -389,25 +295,9 @@ __global__ void __launch_bounds__(kExpandThreads)
   // ---- 1. per-depth lse (float64) and top-k: one warp per depth, one lane per chunk partial
   for (int d = 1 + warp; d <= max_depth; d += kExpandThreads / 32) {
     const RowPartial* rp = part + (static_cast<long long>(b) * max_depth + (d - 1)) * nchunks;
-    float m = -INFINITY;
-    for (int c = lane; c < nchunks; c += 32) m = fmaxf(m, rp[c].m);
-    m = warp_max_f(m);
-    const double md = static_cast<double>(m);
-    double sum = 0.0;
     Cand t[K];
-#pragma unroll
-    for (int i = 0; i < K; ++i) t[i] = Cand{-INFINITY, INT_MAX};
-    for (int c = lane; c < nchunks; c += 32) {
-      sum += rp[c].sum * exp_nonpos_f64(static_cast<double>(rp[c].m) - md, s.tab);
-      Cand u[K];
-#pragma unroll
-      for (int i = 0; i < K; ++i) u[i] = Cand{rp[c].val[i], rp[c].id[i]};
-      merge_k<K>(t, u);
-    }
-    sum = warp_sum_d(sum);
-    warp_merge_k<K>(t, 32);
+    const double lse = warp_merge_row<K>(rp, nchunks, lane, s.tab, t);
     if (lane == 0) {
-      const double lse = md + log(sum);
 #pragma unroll
       for (int r = 0; r < K; ++r) {
         s.lp[d][r] = static_cast<double>(t[r].v) - lse;
@@ -559,21 +449,31 @@ size_t build_workspace_bytes(int batch, int depths, int vocab) {
   return static_cast<size_t>(batch) * depths * nchunks * sizeof(RowPartial);
 }
 
+cudaError_t launch_row_stats(const float* logits, int batch, int rows, int row_stride, int vocab, int topk,
+                             const int32_t* lim_nodes, const int32_t* lim_begin, int lim_budget,
+                             RowPartial* partials, cudaStream_t stream) {
+  const int nchunks = (vocab + kStatsChunk - 1) / kStatsChunk;
+  const dim3 g1(nchunks, batch * rows), b1(build::kThreads);
+  if (topk <= 1)
+    return launch_pdl(build::row_stats_kernel<1>, g1, b1, 0, stream, nullptr, logits, row_stride, vocab, rows,
+                      partials, lim_nodes, lim_begin, lim_budget);
+  if (topk <= 2)
+    return launch_pdl(build::row_stats_kernel<2>, g1, b1, 0, stream, nullptr, logits, row_stride, vocab, rows,
+                      partials, lim_nodes, lim_begin, lim_budget);
+  if (topk <= 4)
+    return launch_pdl(build::row_stats_kernel<4>, g1, b1, 0, stream, nullptr, logits, row_stride, vocab, rows,
+                      partials, lim_nodes, lim_begin, lim_budget);
+  return launch_pdl(build::row_stats_kernel<8>, g1, b1, 0, stream, nullptr, logits, row_stride, vocab, rows,
+                    partials, lim_nodes, lim_begin, lim_budget);
+}
+
 cudaError_t launch_build_tree(const float* logits, const int32_t* root_tokens, int batch, int depths, int vocab,
                               int topk, int budget, int max_depth, int32_t* parent, int32_t* token, float* score,
                               int32_t* depth, RowPartial* partials, int32_t* status, cudaStream_t stream) {
   (void)status;
   const int nchunks = (vocab + kStatsChunk - 1) / kStatsChunk;
-  const dim3 g1(nchunks, batch * max_depth), b1(build::kThreads);
-  cudaError_t e;
-  if (topk <= 1)
-    e = launch_pdl(build::row_stats_kernel<1>, g1, b1, 0, stream, nullptr, logits, depths, vocab, max_depth, partials);
-  else if (topk <= 2)
-    e = launch_pdl(build::row_stats_kernel<2>, g1, b1, 0, stream, nullptr, logits, depths, vocab, max_depth, partials);
-  else if (topk <= 4)
-    e = launch_pdl(build::row_stats_kernel<4>, g1, b1, 0, stream, nullptr, logits, depths, vocab, max_depth, partials);
-  else
-    e = launch_pdl(build::row_stats_kernel<8>, g1, b1, 0, stream, nullptr, logits, depths, vocab, max_depth, partials);
+  cudaError_t e = launch_row_stats(logits, batch, max_depth, depths, vocab, topk, nullptr, nullptr, 0, partials,
+                                   stream);
   if (e != cudaSuccess) return e;
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();

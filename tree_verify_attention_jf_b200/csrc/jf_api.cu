@@ -180,6 +180,50 @@ jf_status jf_build_tree(const float* draft_logits, const int32_t* root_tokens, i
   return JF_OK;
 }
 
+size_t jf_expand_frontier_state_size(int batch, int budget, int topk) {
+  if (batch <= 0 || budget <= 0 || topk <= 0) return 0;
+  return jf::FrontierStateLayout(batch, budget, topk).total;
+}
+
+size_t jf_expand_frontier_workspace_size(int batch, int frontier_rows, int vocab) {
+  if (batch <= 0 || frontier_rows <= 0 || vocab <= 0) return 0;
+  return jf::build_workspace_bytes(batch, frontier_rows, vocab);
+}
+
+jf_status jf_expand_frontier(const float* node_logits, const int32_t* root_tokens, int batch, int frontier_rows,
+                             int vocab, int topk, int budget, int max_depth, int width, int32_t* parent,
+                             int32_t* token, float* score, int32_t* depth, int32_t* num_nodes,
+                             int32_t* frontier_begin, void* state, size_t state_bytes, void* workspace,
+                             size_t workspace_bytes, int32_t* dev_status, jf_stream_t stream) {
+  using namespace jf;
+  if (batch < 0 || frontier_rows <= 0 || vocab <= 0 || topk <= 0 || budget <= 0 || max_depth <= 0 || width <= 0)
+    return JF_ERR_INVALID_ARG;
+  if (topk > kMaxTopk || budget > kMaxFrontierBudget || frontier_rows > kMaxFrontierBudget)
+    return JF_ERR_UNSUPPORTED;
+  if (topk > vocab) return JF_ERR_INVALID_ARG;
+  if (static_cast<long long>(batch) * frontier_rows > 65535) return JF_ERR_UNSUPPORTED;
+  if (batch == 0) return JF_OK;
+  if (!node_logits || !root_tokens || !parent || !token || !score || !depth || !num_nodes || !frontier_begin ||
+      !state || !workspace)
+    return JF_ERR_INVALID_ARG;
+  if (!aligned(node_logits, 4) || !aligned(state, 256) || !aligned(workspace, 16)) return JF_ERR_INVALID_ARG;
+  const FrontierStateLayout lay(batch, budget, topk);
+  if (state_bytes < lay.total) return JF_ERR_INVALID_ARG;
+  if (workspace_bytes < build_workspace_bytes(batch, frontier_rows, vocab)) return JF_ERR_INVALID_ARG;
+  uint8_t* sb = static_cast<uint8_t*>(state);
+  FrontierState st;
+  st.node_key = reinterpret_cast<double*>(sb + lay.key_off);
+  st.cand_lp = reinterpret_cast<double*>(sb + lay.lp_off);
+  st.cand_tok = reinterpret_cast<int32_t*>(sb + lay.tok_off);
+  st.cand_next = reinterpret_cast<int32_t*>(sb + lay.next_off);
+  if (launch_expand_frontier(node_logits, root_tokens, batch, frontier_rows, vocab, topk, budget, max_depth, width,
+                             parent, token, score, depth, num_nodes, frontier_begin, st,
+                             static_cast<RowPartial*>(workspace), dev_status,
+                             reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JF_ERR_CUDA;
+  return JF_OK;
+}
+
 jf_status jf_accept(const int32_t* token, const int32_t* parent, const float* target_logits, int batch,
                     int num_nodes, int vocab, int max_depth, int32_t* accepted_len, int32_t* path,
                     int32_t* bonus_token, int32_t* dev_status, jf_stream_t stream) {

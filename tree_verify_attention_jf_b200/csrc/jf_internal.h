@@ -105,6 +105,41 @@ cudaError_t launch_build_tree(const float* logits, const int32_t* root_tokens, i
                               int topk, int budget, int max_depth, int32_t* parent, int32_t* token, float* score,
                               int32_t* depth, RowPartial* partials, int32_t* status, cudaStream_t stream);
 
+// row statistics of `rows` logits rows per sequence (row stride `row_stride` rows); with lim_nodes / lim_begin
+// only the frontier rows of each sequence whose tree holds fewer than lim_budget nodes are read
+cudaError_t launch_row_stats(const float* logits, int batch, int rows, int row_stride, int vocab, int topk,
+                             const int32_t* lim_nodes, const int32_t* lim_begin, int lim_budget,
+                             RowPartial* partials, cudaStream_t stream);
+
+// ---- frontier expansion from per-node draft logits
+constexpr int kMaxFrontierBudget = 256;  // nodes per tree (= the attention's limit)
+
+struct FrontierState {  // caller-owned, carried from one round to the next
+  double* node_key;     // [B, budget] float64 key of every node
+  double* cand_lp;      // [B, budget, topk] candidate children's log-probabilities
+  int32_t* cand_tok;    // [B, budget, topk] their tokens
+  int32_t* cand_next;   // [B, budget] first untaken rank per node
+};
+
+struct FrontierStateLayout {  // byte offsets in the state buffer, each 256-aligned
+  size_t key_off, lp_off, tok_off, next_off, total;
+  FrontierStateLayout(int batch, int budget, int topk) {
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t nodes = static_cast<size_t>(batch) * budget;
+    key_off = 0;
+    lp_off = up(key_off + nodes * sizeof(double));
+    tok_off = up(lp_off + nodes * topk * sizeof(double));
+    next_off = up(tok_off + nodes * topk * sizeof(int32_t));
+    total = up(next_off + nodes * sizeof(int32_t));
+  }
+};
+
+cudaError_t launch_expand_frontier(const float* logits, const int32_t* root_tokens, int batch, int rows, int vocab,
+                                   int topk, int budget, int max_depth, int width, int32_t* parent, int32_t* token,
+                                   float* score, int32_t* depth, int32_t* num_nodes, int32_t* frontier_begin,
+                                   const FrontierState& st, RowPartial* partials, int32_t* status,
+                                   cudaStream_t stream);
+
 // ---- accept
 constexpr int kMaxAcceptNodes = 1024;
 cudaError_t launch_accept(const int32_t* token, const int32_t* parent, const float* logits, int batch,
