@@ -440,6 +440,62 @@ def build_accept_leg(args, device, capture, timed, pk):
     }
 
 
+def frontier_leg(args, device, flush, pk, batch=8, width=32, topk=4, budget=256, max_depth=16, rounds_before=4):
+    """jf_expand_frontier (per-node draft logits) at batch 8 over the full vocabulary: one round in the middle of a
+    256-node tree (after `rounds_before` rounds, a frontier of `width` nodes), timed from the same saved state each
+    time.  Algorithmic bytes: the frontier rows read once (F x V x 4 per sequence)."""
+    import torch
+
+    from tree_verify_attention_jf_b200 import api, synth
+
+    V = synth.VOCAB
+    roots = torch.arange(1, batch + 1, dtype=torch.int32, device=device)
+    tree = api.FrontierTree(batch, budget, topk, device)
+    gen = torch.Generator(device=device).manual_seed(77)
+    # the draft head's rows for one round: N(0, 2^2) logits (the same random rows every round; each node's own
+    # top-k still comes from the row of its frontier position)
+    logits = torch.randn((batch, width, V), generator=gen, device=device) * 2.0
+    ws = api.expand_frontier_workspace(batch, width, V, device)
+    for _ in range(rounds_before):
+        api.expand_frontier(logits, roots, tree, max_depth, width, workspace=ws)
+    torch.cuda.synchronize()
+    nodes = tree.num_nodes.cpu().tolist()
+    fb = tree.frontier_begin.cpu().tolist()
+    saved = [t.clone() for t in (tree.parent, tree.token, tree.depth, tree.score, tree.num_nodes,
+                                 tree.frontier_begin, tree.state)]
+
+    def restore():
+        for dst, src in zip((tree.parent, tree.token, tree.depth, tree.score, tree.num_nodes, tree.frontier_begin,
+                             tree.state), saved):
+            dst.copy_(src)
+
+    stream = torch.cuda.current_stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        api.expand_frontier(logits, roots, tree, max_depth, width, workspace=ws)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ms = []
+    for it in range(args.steps + 3):
+        restore()
+        flush.zero_()
+        ev[0].record(stream)
+        g.replay()
+        ev[1].record(stream)
+        ev[1].synchronize()
+        if it >= 3:
+            ms.append(ev[0].elapsed_time(ev[1]))
+    del g
+    t = statistics.mean(ms)
+    rows = [n - f for n, f in zip(nodes, fb)]
+    nbytes = sum(rows) * V * 4
+    added = [a - n for a, n in zip(tree.num_nodes.cpu().tolist(), nodes)]
+    return {"call": "jf_expand_frontier", "batch": batch, "vocab": V, "topk": topk, "budget": budget,
+            "width": width, "round": rounds_before + 1, "frontier_rows": rows, "nodes_added": added, "ms": t,
+            "algorithmic_bytes": nbytes, "gbs": nbytes / (t * 1e-3) / 1e9,
+            "hbm_frac": nbytes / (t * 1e-3) / 1e9 / pk["hbm"], "nodes_per_s": sum(added) / (t * 1e-3),
+            "bound": "hbm", "timing": "CUDA graph replay from the saved state, L2 flushed (row statistics + expansion)"}
+
+
 def run_gpu(args, cfg, rank, world, device):
     import torch
 
@@ -586,6 +642,8 @@ def run_gpu(args, cfg, rank, world, device):
                 legs[name] = attention_leg(name, args, device, capture, timed, pk)
                 torch.cuda.empty_cache()
         legs.update(build_accept_leg(args, device, capture, timed, pk))
+        torch.cuda.empty_cache()
+        legs["expand_frontier"] = frontier_leg(args, device, flush, pk)
         torch.cuda.empty_cache()
         r["legs"] = legs
     return r
