@@ -17,9 +17,10 @@
 //     PV and next QK.
 //   * Per CTA (12 warps): warp 0 loads Q (double-buffered, once per segment) and gathers this CTA's half of
 //     every K tile, warp 2 its half of every V tile -- one TMA box per page and 64-column half, 128-byte
-//     swizzled, gathered through the block table.  Each copy lands on a barrier of its own CTA; the warp
-//     then zeroes V rows past the sequence end and hands the tile on to the even CTA's MMA warp with one
-//     cluster-scope arrival.  Warp 1 allocates the pair's tensor memory and (in the even CTA) issues the
+//     swizzled, gathered through the block table, in a 4-deep ring.  The copies are CTA-pair TMA loads: each
+//     lands in its own CTA's shared memory and completes its bytes on the even CTA's barrier.  V rows past
+//     the sequence end are zeroed (a partial last page lands on a barrier of its own CTA first) before the
+//     CTA's arrival on the even CTA's barrier.  Warp 1 allocates the pair's tensor memory and (in the even CTA) issues the
 //     MMAs; every commit is multicast to both CTAs' barriers.  Warp 3 validates each segment's metadata.
 //     Warps 4-11 are two softmax warpgroups: the thread of warpgroup h for row r owns columns
 //     [64 h, 64 h + 64) of that row; the two exchange their row maxima through shared memory once per
@@ -34,9 +35,10 @@
 //     dependency, merges each recorded unit's partials and stores the bf16 output.  Nothing spins on
 //     another CTA pair.
 //   * Every wait is bounded (a %globaltimer limit); a role that gives up reports JF_ERR_TIMEOUT, raises
-//     its CTA's and the peer CTA's abort flag, and every role then unwinds to the common exit, where the
-//     copy warps wait (bounded) for the copies they issued and the MMA warp for its last MMA before the
-//     pair's tensor memory is released.
+//     its CTA's and the peer CTA's abort flag, and every role then unwinds to the common exit: the copy
+//     warps first wait long enough for every copy they issued to land, the MMA warp for its last MMA, and
+//     the softmax warps keep meeting their shared barriers with their work skipped, so that the pair's
+//     tensor memory is released only when nothing can still write it.
 #include "jf_device.cuh"
 #include "jf_internal.h"
 
@@ -47,7 +49,7 @@ constexpr int kPage = 16;
 constexpr int kBM = 128;             // rows per CTA (the pair's M tile is 2 x kBM)
 constexpr int kBN = 128;             // keys per KV tile
 constexpr int kPagesPerTile = kBN / kPage;
-constexpr int kStages = 3;           // K and V ring depth
+constexpr int kStages = 4;           // K and V ring depth
 constexpr int kSBufs = 3;            // S ring depth in tensor memory
 constexpr int kThreads = 384;
 constexpr int kQHalf = kBM * 128;                 // 128 rows x 64 bf16
@@ -75,10 +77,13 @@ struct __align__(1024) Smem {
   long long scan_warp[kThreads / 32];
   float red[2][2][kBM];   // row maxima of the two softmax warpgroups, by tile parity
   float lsum[2][kBM];     // row sums of the two softmax warpgroups at a segment's end
-  uint64_t qland[2], qfull[2], qempty[2];
-  uint64_t kland[kStages], kfull[kStages], kempty[kStages];
-  uint64_t vland[kStages], vfull[kStages], vempty[kStages];
-  uint64_t sfull[kSBufs], pfull[kSBufs], pvdone, drain;
+  uint64_t qfull[2], qempty[2];
+  uint64_t kfull[kStages], kempty[kStages];
+  uint64_t vfull[kStages], vempty[kStages];
+  // S, P and PV of tile i use entry i % 3: a waiter is never more than one phase behind (tile i - 3 has
+  // completed before tile i is waited for), so parity waits are unambiguous
+  uint64_t sfull[kSBufs], pfull[kSBufs], pvdone[kSBufs], drain;
+  uint64_t vpart;  // this CTA's copy of a partial last page of V
   uint64_t metafull[2], metaempty[2];
   uint32_t tmem_base;
   int meta_valid[2];
@@ -226,74 +231,36 @@ __device__ __forceinline__ int batch_page_ids(const AttnParams& p, const int32_t
 }
 
 // ------------------------------------------------------------------------------------------------
-// Warp 0: Q (double-buffered, one load per segment) and this CTA's half of every K tile.  Warp 2: this
-// CTA's 64 head dims of every V tile.  Each tile lands on a barrier of this CTA; the warp hands it on to
-// the even CTA's MMA warp one tile later (after issuing the next tile), so the copies stay in flight.
+// Warp 0: Q (double-buffered, one load per segment) and this CTA's 64 keys of every K tile.  Warp 2: this
+// CTA's 64 head dims of every V tile.  Every copy is a CTA-pair TMA: it lands in this CTA's shared memory and
+// completes its bytes on the even CTA's barrier, which the even CTA's copy warp arms with the bytes of both
+// CTAs (one arrival); for V, the odd CTA adds one arrival of its own (vfull counts 2), made after it has
+// zeroed its stage's rows past the sequence end.
 // ------------------------------------------------------------------------------------------------
-struct Relay {  // a landed-but-not-yet-handed-on tile
-  int stage, zf;  // stage; first row past the sequence (V only; kBN = none)
-  uint32_t parity;
-  bool live;
-};
-
-// Copies a producer warp has issued and not yet seen land: on an abort the warp waits for them (bounded)
-// before the CTA may exit, so that no copy writes into the shared memory of an exited CTA.
-struct InFlight {
-  uint32_t stages;   // bit i: stage i of the K (or V) ring
-  uint32_t parity;   // bit i: the phase parity stage i's copy completes
-  uint32_t q;        // bit i: Q buffer i
-  uint32_t qparity;  // bit i: the phase parity Q buffer i's copy completes
-};
-
+// Once a copy warp has given up it waits this long before its CTA may exit, so that every copy it issued
+// has landed (copies take microseconds).
+constexpr uint64_t kDrainNs = 200000ull;  // 200 us
+__device__ __forceinline__ void drain_delay() {
+  const uint64_t t0 = globaltimer();
+  while (globaltimer() - t0 < kDrainNs) __nanosleep(1000);
+}
 // Waits up to `ns` for a phase, ignoring the abort flag (used only while unwinding).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t ns) {
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(bar, parity))
     if (globaltimer() - t0 > ns) return;
 }
-constexpr uint64_t kDrainNs = 50000000ull;  // 50 ms
 
 __device__ bool kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_v, uint32_t rank,
-                            const CUtensorMap* tm_q, const CUtensorMap* tm_kv, InFlight& fl) {
+                            const CUtensorMap* tm_q, const CUtensorMap* tm_kv) {
   const int lane = threadIdx.x & 31;
   volatile int* abort = &s.abort_flag;
-  uint64_t* land = is_v ? s.vland : s.kland;
   uint64_t* empty = is_v ? s.vempty : s.kempty;
   const uint32_t full0 = mapa_shared(smem_u32(is_v ? s.vfull : s.kfull), 0);  // the even CTA's full barriers
   const uint32_t qfull0 = mapa_shared(smem_u32(s.qfull), 0);
   Seg g;
-  uint32_t it = 0, sidx = 0;
+  uint32_t it = 0, sidx = 0, vpart_uses = 0;
   const int nodes_per_half = kBM / p.group;
-  Relay pend{0, kBN, 0u, false};
-  Relay qpend{0, 0, 0u, false};
-  fl.stages = fl.parity = fl.q = fl.qparity = 0;
-  auto hand_on = [&](Relay& r) -> bool {  // wait for the tile to land here, fix it up, signal the even CTA
-    if (!r.live) return true;
-    if (!warp_wait(&land[r.stage], r.parity, abort)) return false;
-    fl.stages &= ~(1u << r.stage);
-    if (is_v && r.zf < kBN) {
-      // Keys beyond the sequence's last slot: clear their V rows so stale cache contents (even NaN) cannot
-      // reach the output through 0 * V.  Whole 128-byte rows are cleared, so the swizzle does not matter.
-      uint8_t* vb = s.v[r.stage];
-      const int z0 = r.zf < 0 ? 0 : r.zf;
-      for (int i = lane; i < (kBN - z0) * 8; i += 32)
-        *reinterpret_cast<uint4*>(vb + (z0 + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
-      fence_proxy_async_smem();
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(full0 + r.stage * 8);
-    r.live = false;
-    return true;
-  };
-  auto hand_on_q = [&]() -> bool {
-    if (!qpend.live) return true;
-    if (!warp_wait(&s.qland[qpend.stage], qpend.parity, abort)) return false;
-    fl.q &= ~(1u << qpend.stage);
-    __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(qfull0 + qpend.stage * 8);
-    qpend.live = false;
-    return true;
-  };
   while (iter.next(s, p, g)) {
     const int npg = (g.P + g.N + kPage - 1) / kPage;
     const int32_t* bt = p.block_table + static_cast<long long>(g.b) * p.max_pages;
@@ -302,15 +269,12 @@ __device__ bool kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
     if (!is_v) {  // this CTA's 128 Q rows go out while the page ids are on their way
       const int qb = sidx & 1;
       if (!warp_wait(&s.qempty[qb], ((sidx >> 1) & 1) ^ 1, abort)) return false;
-      if (lane == 0) mbar_arrive_expect_tx(&s.qland[qb], kQBytes);
+      if (rank == 0 && lane == 0) mbar_arrive_expect_tx_cluster(qfull0 + qb * 8, 2 * kQBytes);
       __syncwarp();
       if (lane < 2) {
         const int node0 = g.off + (g.mp * 2 + static_cast<int>(rank)) * nodes_per_half;
-        tma_load_3d(s.q[qb] + lane * kQHalf, tm_q, &s.qland[qb], lane * 64, g.kvh * p.group, node0);
+        tma_load_3d_pair(s.q[qb] + lane * kQHalf, tm_q, qfull0 + qb * 8, lane * 64, g.kvh * p.group, node0);
       }
-      fl.q |= 1u << qb;
-      fl.qparity = (fl.qparity & ~(1u << qb)) | (((sidx >> 1) & 1u) << qb);
-      qpend = Relay{qb, 0, (sidx >> 1) & 1, true};
     }
     for (int t = g.kb; t < g.ke; ++t, ++it) {
       const int st = it % kStages;
@@ -320,13 +284,7 @@ __device__ bool kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
         ids_cur = ids_next;
         ids_next = batch_page_ids(p, bt, npg, t + 4, g.ke, lane);
       }
-      // K: lane j < 8 copies page 4 * rank + j / 2 of the tile, 64-dim half j % 2 (this CTA's 64 keys);
-      // V: lane j < 8 copies page j of the tile, this CTA's 64 dims
-      const int page = is_v ? (lane & 7) : (4 * static_cast<int>(rank) + ((lane >> 1) & 3));
-      int pid = __shfl_sync(0xffffffffu, ids_cur, bi * 8 + page);
-      if (lane >= 8) pid = -1;
-      const uint32_t mask = __ballot_sync(0xffffffffu, pid >= 0);
-      const uint32_t bytes = static_cast<uint32_t>(__popc(mask)) * (kPage * 128u);
+      const uint32_t bar = full0 + st * 8;
       if (!warp_wait(&empty[st], ph ^ 1, abort)) return false;
       if (is_v && it == 0) {
         // The copy engine serves requests in order and the first S needs Q and K only: the kernel's
@@ -336,41 +294,64 @@ __device__ bool kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
           if (*abort || globaltimer() - t0 > kWaitLimitNs) return false;
         }
       }
-      if (lane == 0) mbar_arrive_expect_tx(&land[st], bytes);
-      __syncwarp();
-      if (pid >= 0) {
-        if (is_v) {
-          tma_load_3d(s.v[st] + lane * (kPage * 128), tm_kv, &land[st], static_cast<int>(rank) * 64, g.kvh,
-                      pid * kPage);
-        } else {
+      if (!is_v) {
+        // lane j < 8 copies page 4 * rank + j / 2 of the tile, 64-dim half j % 2 (this CTA's 64 keys); the even
+        // CTA arms the barrier with the bytes of all the tile's pages (both CTAs).  Keys past the sequence
+        // are not copied: their S columns are masked before the softmax.
+        const int pid_all = __shfl_sync(0xffffffffu, ids_cur, bi * 8 + (lane & 7));
+        const uint32_t all = __ballot_sync(0xffffffffu, lane < 8 && pid_all >= 0);
+        int pid = __shfl_sync(0xffffffffu, ids_cur, bi * 8 + 4 * static_cast<int>(rank) + ((lane >> 1) & 3));
+        if (rank == 0 && lane == 0) mbar_arrive_expect_tx_cluster(bar, static_cast<uint32_t>(__popc(all)) * 4096u);
+        if (lane < 8 && pid >= 0) {
           const int half = lane & 1;
-          tma_load_3d(s.k[st] + half * kKHalf + (lane >> 1) * (kPage * 128), tm_kv, &land[st], half * 64, g.kvh,
-                      pid * kPage);
+          tma_load_3d_pair(s.k[st] + half * kKHalf + (lane >> 1) * (kPage * 128), tm_kv, bar, half * 64, g.kvh,
+                           pid * kPage);
+        }
+        if (it == 0) {
+          __syncwarp();
+          if (lane == 0) *reinterpret_cast<volatile int*>(&s.k_started) = 1;
+        }
+      } else {
+        // V rows of the tile past the sequence end are zeroed so that stale cache contents (even NaN) cannot
+        // reach the output through 0 * V.  Full pages are CTA-pair copies; the sequence's last page, if
+        // partial, is copied to this CTA alone (a barrier of its own), and the warp waits for it, zeroes the
+        // rows past the end and only then arrives on the even CTA's barrier.
+        const int nkeys = g.P + g.N - t * kBN;
+        const int zf = nkeys < 0 ? 0 : (nkeys > kBN ? kBN : nkeys);
+        const int full_pages = zf / kPage, part = zf % kPage;
+        const int pid = __shfl_sync(0xffffffffu, ids_cur, bi * 8 + (lane & 7));
+        const bool full_ok = lane < full_pages && pid >= 0;  // full_pages <= 8
+        const int pid_part = __shfl_sync(0xffffffffu, ids_cur, bi * 8 + (full_pages & 7));
+        const bool part_ok = part > 0 && pid_part >= 0;
+        const uint32_t nfull = static_cast<uint32_t>(__popc(__ballot_sync(0xffffffffu, full_ok)));
+        if (full_ok)
+          tma_load_3d_pair(s.v[st] + lane * (kPage * 128), tm_kv, bar, static_cast<int>(rank) * 64, g.kvh,
+                           pid * kPage);
+        if (part_ok) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&s.vpart, kPage * 128);
+            tma_load_3d(s.v[st] + full_pages * (kPage * 128), tm_kv, &s.vpart, static_cast<int>(rank) * 64,
+                        g.kvh, pid_part * kPage);
+          }
+          if (!warp_wait(&s.vpart, vpart_uses & 1, abort)) return false;
+          ++vpart_uses;
+        }
+        if (zf < kBN) {
+          uint8_t* vb = s.v[st];
+          for (int i = lane; i < (kBN - zf) * 8; i += 32)
+            *reinterpret_cast<uint4*>(vb + (zf + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive_expect_tx_cluster(bar, 2 * nfull * (kPage * 128u));  // both CTAs' full pages
+          else mbar_arrive_cluster(bar);
         }
       }
-      fl.stages |= 1u << st;
-      fl.parity = (fl.parity & ~(1u << st)) | (ph << st);
-      if (!is_v && it == 0) {
-        __syncwarp();
-        if (lane == 0) *reinterpret_cast<volatile int*>(&s.k_started) = 1;
-      }
-      // hand on the previous tile, then (first tile of a segment) the segment's Q
-      if (!hand_on(pend)) return false;
-      pend = Relay{st, g.P + g.N - t * kBN, ph, true};
-      if (!is_v && t == g.kb && !hand_on_q()) return false;
     }
     ++sidx;
   }
-  return hand_on(pend);
-}
-
-// After an abort: wait (bounded) for every copy this warp issued and has not seen land.
-__device__ void drain_copies(Smem& s, bool is_v, const InFlight& fl) {
-  uint64_t* land = is_v ? s.vland : s.kland;
-  for (int st = 0; st < kStages; ++st)
-    if (fl.stages & (1u << st)) drain_wait(&land[st], (fl.parity >> st) & 1u, kDrainNs);
-  for (int qb = 0; qb < 2; ++qb)
-    if (fl.q & (1u << qb)) drain_wait(&s.qland[qb], (fl.qparity >> qb) & 1u, kDrainNs);
+  return true;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -445,7 +426,7 @@ __device__ bool mma_issuer(Smem& s, const AttnParams& p, SegIter pv_iter, uint32
       if (lane == 0) {
         issue_pv(s, tmem, sb, st, t == gp.kb);
         mma2_commit_mc(&s.vempty[st], kPairMask);
-        mma2_commit_mc(&s.pvdone, kPairMask);
+        mma2_commit_mc(&s.pvdone[sb], kPairMask);
       }
       __syncwarp();
       issued = true;
@@ -678,7 +659,7 @@ __device__ bool softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
       }
       if (__any_sync(0xffffffffu, resc)) {
         // O holds PV of the segment's tiles so far; the last of them (tile it - 1) may still be running
-        if (!warp_wait(&s.pvdone, (it - 1) & 1, abort)) {
+        if (!warp_wait(&s.pvdone[(it - 1) % kSBufs], ((it - 1) / kSBufs) & 1, abort)) {
           ok = false;
           continue;
         }
@@ -731,7 +712,7 @@ __device__ bool softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
     if (ok && !warp_wait(&s.metafull[buf], (sidx >> 1) & 1, abort)) ok = false;
     if (ok) {
       seg_ok = s.meta_valid[buf] != 0;
-      if (!warp_wait(&s.pvdone, (it - 1) & 1, abort)) ok = false;  // the segment's last PV
+      if (!warp_wait(&s.pvdone[(it - 1) % kSBufs], ((it - 1) / kSBufs) & 1, abort)) ok = false;  // last PV
     }
     if (ok) {
       tc_fence_after();
@@ -807,26 +788,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   // peer CTA before any arrival crosses over.
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.qland[i], 1);
-      mbar_init(&s.qfull[i], 2);
+      mbar_init(&s.qfull[i], 1);
       mbar_init(&s.qempty[i], 1);
       mbar_init(&s.metafull[i], 32);
       mbar_init(&s.metaempty[i], kSoftmaxThreads);
     }
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&s.kland[i], 1);
-      mbar_init(&s.kfull[i], 2);
+      mbar_init(&s.kfull[i], 1);  // the even CTA's arrival (with both CTAs' bytes)
       mbar_init(&s.kempty[i], 1);
-      mbar_init(&s.vland[i], 1);
-      mbar_init(&s.vfull[i], 2);
+      mbar_init(&s.vfull[i], 2);  // both CTAs' arrivals (the even CTA's with both CTAs' bytes)
       mbar_init(&s.vempty[i], 1);
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&s.sfull[i], 1);
       mbar_init(&s.pfull[i], kPfullCount);
+      mbar_init(&s.pvdone[i], 1);
     }
-    mbar_init(&s.pvdone, 1);
     mbar_init(&s.drain, 1);
+    mbar_init(&s.vpart, 1);
     s.abort_flag = 0;
     s.k_started = 0;
     fence_barrier_init();
@@ -872,10 +851,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       iter.b = lo;
     }
     if (warp == 0 || warp == 2) {
-      InFlight fl;
-      if (!kv_producer(s, p, iter, warp == 2, rank, &tm_q, warp == 2 ? &tm_v : &tm_k, fl)) {
+      if (!kv_producer(s, p, iter, warp == 2, rank, &tm_q, warp == 2 ? &tm_v : &tm_k)) {
         set_abort(s, p);
-        drain_copies(s, warp == 2, fl);
+        drain_delay();
       }
     } else if (warp == 1) {
       if (rank == 0) {
