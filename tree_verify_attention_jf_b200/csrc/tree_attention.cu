@@ -62,10 +62,10 @@ constexpr uint32_t kTmO = 384;                    // O at column 384, S_i at 128
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow up to 2^8 before O is rescaled
 constexpr int kSegCost = 3;  // kv tiles' worth of time that starting a segment in mid-kernel costs
 constexpr int kSoftmaxThreads = 2 * kBM;
-// P-ready: one arrival per softmax warp of the even CTA plus one forwarded from the odd CTA (whose warps
-// arrive on a barrier of their own; its warp 1 turns that into one cluster-scope arrival, so the softmax
-// warps never pay for a cluster-scope release)
-constexpr uint32_t kPfullCount = kSoftmaxThreads / 32 + 1;
+// P-ready: one arrival per softmax warp of both CTAs.  The odd CTA's are relaxed cluster-scope arrivals: P sits
+// in tensor memory, its stores complete (tcgen05.wait::st) before the arrival, and a release at cluster scope
+// would cost each softmax warp a membar per tile.
+constexpr uint32_t kPfullCount = 2 * (kSoftmaxThreads / 32);
 constexpr uint16_t kPairMask = 0x3;
 
 struct __align__(1024) Smem {
@@ -85,7 +85,7 @@ struct __align__(1024) Smem {
   uint64_t vfull[kStages], vempty[kStages];
   // S, P and PV of tile i use entry i % 3: a waiter is never more than one phase behind (tile i - 3 has
   // completed before tile i is waited for), so parity waits are unambiguous
-  uint64_t sfull[kSBufs], pfull[kSBufs], pvdone[kSBufs], pdone[kSBufs], drain;
+  uint64_t sfull[kSBufs], pfull[kSBufs], pvdone[kSBufs], drain;
   uint64_t vpart;  // this CTA's copy of a partial last page of V
   uint64_t metafull[2], metaempty[2];
   uint32_t tmem_base;
@@ -348,7 +348,8 @@ __device__ bool kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
         __syncwarp();
         if (lane == 0) {
           if (rank == 0) mbar_arrive_expect_tx(&s.vfull[st], 2 * nfull * (kPage * 128u));  // both CTAs' pages
-          else mbar_arrive_cluster(bar);
+          else if (zf < kBN) mbar_arrive_cluster(bar);  // publishes the zeroed rows (release)
+          else mbar_arrive_cluster_relaxed(bar);        // the copies complete on the barrier themselves
         }
       }
     }
@@ -434,25 +435,6 @@ __device__ bool mma_issuer(Smem& s, const AttnParams& p, SegIter pv_iter, uint32
       __syncwarp();
       issued = true;
       if (!issue_next_qk()) return false;
-    }
-  }
-  return true;
-}
-
-// ------------------------------------------------------------------------------------------------
-// Warp 1 of the odd CTA: forwards each tile's P-ready (this CTA's 8 softmax warps, counted on pdone) to the even
-// CTA's barrier with one cluster-scope arrival.
-// ------------------------------------------------------------------------------------------------
-__device__ bool p_forwarder(Smem& s, const AttnParams& p, SegIter iter) {
-  volatile int* abort = &s.abort_flag;
-  const uint32_t pfull0 = mapa_shared(smem_u32(s.pfull), 0);
-  Seg g;
-  uint32_t it = 0;
-  while (iter.next(s, p, g)) {
-    for (int t = g.kb; t < g.ke; ++t, ++it) {
-      const int sb = it % kSBufs;
-      if (!warp_wait(&s.pdone[sb], (it / kSBufs) & 1, abort)) return false;
-      if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(pfull0 + sb * 8);
     }
   }
   return true;
@@ -614,6 +596,7 @@ __device__ bool softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
   const int wq = (threadIdx.x >> 5) & 3;
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
   volatile int* abort = &s.abort_flag;
+  const uint32_t pfull0 = mapa_shared(smem_u32(s.pfull), 0);  // the even CTA's P-ready barriers
   const float sl2 = p.scale_log2;
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
   const int nodes_per_half = kBM / p.group;
@@ -726,7 +709,10 @@ __device__ bool softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive(rank == 0 ? &s.pfull[sb] : &s.pdone[sb]);
+      if ((threadIdx.x & 31) == 0) {
+        if (rank == 0) mbar_arrive(&s.pfull[sb]);
+        else mbar_arrive_cluster_relaxed(pfull0 + sb * 8);
+      }
     }
     // ---------------- epilogue of the segment
     bool seg_ok = false;
@@ -824,7 +810,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.sfull[i], 1);
       mbar_init(&s.pfull[i], kPfullCount);
       mbar_init(&s.pvdone[i], 1);
-      mbar_init(&s.pdone[i], kSoftmaxThreads / 32);
     }
     mbar_init(&s.drain, 1);
     mbar_init(&s.vpart, 1);
@@ -878,9 +863,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_delay();
       }
     } else if (warp == 1) {
-      if (rank == 1) {
-        if (!p_forwarder(s, p, iter)) set_abort(s, p);
-      } else {
+      if (rank == 0) {
         bool issued = false;
         if (!mma_issuer(s, p, iter, tmem, issued)) {
           set_abort(s, p);
