@@ -360,7 +360,10 @@ __device__ bool kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
 
 // ------------------------------------------------------------------------------------------------
 // Warp 1 of the even CTA: CTA-pair tcgen05.mma issuer.  QK of tile i goes into S buffer i % 3 and is issued
-// right after PV of tile i - 3 (which read P from that buffer); every commit is multicast to both CTAs.
+// right after PV of tile i - 3 (which read P from that buffer); every commit is multicast to both CTAs.  Its
+// waits acquire at CTA scope (a cluster-scope acquire costs hundreds of cycles per wait on this critical
+// warp): the odd CTA's P-ready arrivals are relaxed (P is in tensor memory, its stores complete before the
+// arrival) and the copies' bytes complete on the barriers themselves.
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ void issue_qk(const Smem& s, uint32_t tmem, int qb, int st, int sb) {
   constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, false, false);
@@ -403,8 +406,8 @@ __device__ bool mma_issuer(Smem& s, const AttnParams& p, SegIter pv_iter, uint32
     }
     const int qb = qk_sidx & 1;
     const int st = it_qk % kStages;
-    if (qk_t == gq.kb && !warp_wait_cluster(&s.qfull[qb], (qk_sidx >> 1) & 1, abort)) return false;
-    if (!warp_wait_cluster(&s.kfull[st], (it_qk / kStages) & 1, abort)) return false;
+    if (qk_t == gq.kb && !warp_wait(&s.qfull[qb], (qk_sidx >> 1) & 1, abort)) return false;
+    if (!warp_wait(&s.kfull[st], (it_qk / kStages) & 1, abort)) return false;
     tc_fence_after();
     if (lane == 0) {
       issue_qk(s, tmem, qb, st, it_qk % kSBufs);
@@ -424,8 +427,13 @@ __device__ bool mma_issuer(Smem& s, const AttnParams& p, SegIter pv_iter, uint32
   while (pv_iter.next(s, p, gp)) {
     for (int t = gp.kb; t < gp.ke; ++t, ++it) {
       const int sb = it % kSBufs, st = it % kStages;
-      if (!warp_wait_cluster(&s.pfull[sb], (it / kSBufs) & 1, abort)) return false;
-      if (!warp_wait_cluster(&s.vfull[st], (it / kStages) & 1, abort)) return false;
+      if (!warp_wait(&s.pfull[sb], (it / kSBufs) & 1, abort)) return false;
+      // Cluster scope only for the tile whose V rows past the sequence end the odd CTA zeroed (its arrival is a
+      // release); every other arrival is relaxed or local, and the copies' bytes complete on the barrier.
+      const bool zeroed = static_cast<long long>(t + 1) * kBN > static_cast<long long>(gp.P) + gp.N;
+      if (!(zeroed ? warp_wait_cluster(&s.vfull[st], (it / kStages) & 1, abort)
+                   : warp_wait(&s.vfull[st], (it / kStages) & 1, abort)))
+        return false;
       tc_fence_after();
       if (lane == 0) {
         issue_pv(s, tmem, sb, st, t == gp.kb);
