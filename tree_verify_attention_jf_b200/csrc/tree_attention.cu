@@ -386,17 +386,21 @@ __device__ __forceinline__ void issue_pv(const Smem& s, uint32_t tmem, int sb, i
   }
 }
 
+// Only lane 0 runs the issue loop (the other lanes wait at the warp's exit).  Per tile it waits for everything
+// the tile's burst needs -- P and V of tile i, K (and at a segment start Q) of tile i + 3 -- and then issues PV(i)
+// and QK(i + 3) back to back, so that the tensor pipe is fed 16 MMAs at a time.
 __device__ bool mma_issuer(Smem& s, const AttnParams& p, SegIter pv_iter, uint32_t tmem, bool& issued) {
-  const int lane = threadIdx.x & 31;
   volatile int* abort = &s.abort_flag;
   issued = false;
-  // the QK side runs up to kSBufs tiles ahead of the PV side on its own copy of the segment iterator
+  // the QK side runs kSBufs tiles ahead of the PV side on its own copy of the segment iterator
   SegIter qk_iter = pv_iter;
   Seg gq, gp;
   bool qk_live = qk_iter.next(s, p, gq);
   int qk_t = qk_live ? gq.kb : 0;
   uint32_t it_qk = 0, qk_sidx = 0;
-  auto issue_next_qk = [&]() -> bool {
+  // Waits for the next QK's operands; false on a timeout/abort.  *have = false when no QK is left.
+  auto wait_next_qk = [&](bool* have) -> bool {
+    *have = false;
     if (!qk_live) return true;
     if (qk_t == gq.ke) {
       ++qk_sidx;
@@ -404,45 +408,47 @@ __device__ bool mma_issuer(Smem& s, const AttnParams& p, SegIter pv_iter, uint32
       if (!qk_live) return true;
       qk_t = gq.kb;
     }
-    const int qb = qk_sidx & 1;
-    const int st = it_qk % kStages;
-    if (qk_t == gq.kb && !warp_wait(&s.qfull[qb], (qk_sidx >> 1) & 1, abort)) return false;
-    if (!warp_wait(&s.kfull[st], (it_qk / kStages) & 1, abort)) return false;
-    tc_fence_after();
-    if (lane == 0) {
-      issue_qk(s, tmem, qb, st, it_qk % kSBufs);
-      mma2_commit_mc(&s.sfull[it_qk % kSBufs], kPairMask);
-      mma2_commit_mc(&s.kempty[st], kPairMask);
-      if (qk_t == gq.ke - 1) mma2_commit_mc(&s.qempty[qb], kPairMask);
-    }
-    __syncwarp();
-    issued = true;
-    ++qk_t;
-    ++it_qk;
+    if (qk_t == gq.kb && !mbar_wait(&s.qfull[qk_sidx & 1], (qk_sidx >> 1) & 1, abort)) return false;
+    if (!mbar_wait(&s.kfull[it_qk % kStages], (it_qk / kStages) & 1, abort)) return false;
+    *have = true;
     return true;
   };
-  for (int i = 0; i < kSBufs; ++i)
-    if (!issue_next_qk()) return false;
+  auto issue_qk_now = [&]() {
+    const int qb = qk_sidx & 1, st = it_qk % kStages;
+    issue_qk(s, tmem, qb, st, it_qk % kSBufs);
+    mma2_commit_mc(&s.sfull[it_qk % kSBufs], kPairMask);
+    mma2_commit_mc(&s.kempty[st], kPairMask);
+    if (qk_t == gq.ke - 1) mma2_commit_mc(&s.qempty[qb], kPairMask);
+    ++qk_t;
+    ++it_qk;
+    issued = true;
+  };
+  for (int i = 0; i < kSBufs; ++i) {
+    bool have;
+    if (!wait_next_qk(&have)) return false;
+    if (!have) break;
+    tc_fence_after();
+    issue_qk_now();
+  }
   uint32_t it = 0;
   while (pv_iter.next(s, p, gp)) {
     for (int t = gp.kb; t < gp.ke; ++t, ++it) {
       const int sb = it % kSBufs, st = it % kStages;
-      if (!warp_wait(&s.pfull[sb], (it / kSBufs) & 1, abort)) return false;
+      if (!mbar_wait(&s.pfull[sb], (it / kSBufs) & 1, abort)) return false;
       // Cluster scope only for the tile whose V rows past the sequence end the odd CTA zeroed (its arrival is a
       // release); every other arrival is relaxed or local, and the copies' bytes complete on the barrier.
       const bool zeroed = static_cast<long long>(t + 1) * kBN > static_cast<long long>(gp.P) + gp.N;
-      if (!(zeroed ? warp_wait_cluster(&s.vfull[st], (it / kStages) & 1, abort)
-                   : warp_wait(&s.vfull[st], (it / kStages) & 1, abort)))
+      if (!(zeroed ? mbar_wait_cluster(&s.vfull[st], (it / kStages) & 1, abort)
+                   : mbar_wait(&s.vfull[st], (it / kStages) & 1, abort)))
         return false;
+      bool have;
+      if (!wait_next_qk(&have)) return false;
       tc_fence_after();
-      if (lane == 0) {
-        issue_pv(s, tmem, sb, st, t == gp.kb);
-        mma2_commit_mc(&s.vempty[st], kPairMask);
-        mma2_commit_mc(&s.pvdone[sb], kPairMask);
-      }
-      __syncwarp();
+      issue_pv(s, tmem, sb, st, t == gp.kb);
+      mma2_commit_mc(&s.vempty[st], kPairMask);
+      mma2_commit_mc(&s.pvdone[sb], kPairMask);
       issued = true;
-      if (!issue_next_qk()) return false;
+      if (have) issue_qk_now();
     }
   }
   return true;
@@ -871,18 +877,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_delay();
       }
     } else if (warp == 1) {
-      if (rank == 0) {
+      if (rank == 0 && (tid & 31) == 0) {
         bool issued = false;
         if (!mma_issuer(s, p, iter, tmem, issued)) {
           set_abort(s, p);
-          if (issued && (tid & 31) == 0) {
+          if (issued) {
             // the pair's tensor memory is released only after the last MMA issued has completed
             mma2_commit_mc(&s.drain, 0x1);
             drain_wait(&s.drain, 0, kDrainNs);
           }
-          __syncwarp();
         }
       }
+      __syncwarp();
     } else if (warp == 3) {
       if (!metadata(s, p, iter)) set_abort(s, p);
     } else {
