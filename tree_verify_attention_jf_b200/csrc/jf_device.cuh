@@ -381,4 +381,10 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Arrives on named barrier `id` without waiting (the producer side of a producer/consumer hand-off: shared
+// memory written before the arrival is visible to the threads that complete a bar.sync on it).
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 }  // namespace jf

@@ -62,10 +62,10 @@ constexpr uint32_t kTmO = 384;                    // O at column 384, S_i at 128
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow up to 2^8 before O is rescaled
 constexpr int kSegCost = 3;  // kv tiles' worth of time that starting a segment in mid-kernel costs
 constexpr int kSoftmaxThreads = 2 * kBM;
-// P-ready: one arrival per softmax warp of both CTAs.  The odd CTA's are relaxed cluster-scope arrivals: P sits
+// P-ready: one arrival per warp of the tile's softmax warpgroup in both CTAs.  The odd CTA's are relaxed cluster-scope arrivals: P sits
 // in tensor memory, its stores complete (tcgen05.wait::st) before the arrival, and a release at cluster scope
 // would cost each softmax warp a membar per tile.
-constexpr uint32_t kPfullCount = 2 * (kSoftmaxThreads / 32);
+constexpr uint32_t kPfullCount = 2 * (kSoftmaxThreads / 64);  // the 4 warps of one warpgroup, both CTAs
 constexpr uint16_t kPairMask = 0x3;
 
 struct __align__(1024) Smem {
@@ -78,8 +78,9 @@ struct __align__(1024) Smem {
   int seq_p[kMaxAttnBatch];        // prefix length of every sequence (copied once by the plan)
   int seq_off[kMaxAttnBatch + 1];  // tree_offsets
   long long scan_warp[kThreads / 32];
-  float red[2][2][kBM];   // row maxima of the two softmax warpgroups, by tile parity
-  float lsum[2][kBM];     // row sums of the two softmax warpgroups at a segment's end
+  float mhand[2][kBM];    // the running maximum decided at a tile, by tile parity, for the next tile's owner
+  float lsum[2][2][kBM];  // row sums of the two softmax warpgroups at a segment's end (by segment parity)
+  float msum[2][2][kBM];  // the running maximum each warpgroup's row sum is under
   uint64_t qfull[2], qempty[2];
   uint64_t kfull[kStages], kempty[kStages];
   uint64_t vfull[kStages], vempty[kStages];
@@ -602,10 +603,72 @@ __device__ bool build_ancestors(Smem& s, const AttnParams& p, const Seg& g) {
   return true;
 }
 
-// A warp whose wait gives up keeps running the loop structure with its work skipped (ok = false), so that
-// the named barriers the 256 softmax threads share are always reached by all of them.
+// S columns [c0, c0 + 64) of the row into sr, with the tree mask applied (invisible keys -> -inf); returns
+// their maximum (raw scores).
+__device__ __forceinline__ float load_masked_half(uint32_t taddr, uint32_t (&sr)[64], bool tree_tile, int slot0,
+                                                  const Seg& g, bool row_valid, const uint32_t* anc) {
+  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+  uint32_t vis[2];
+#pragma unroll
+  for (int w = 0; w < 2; ++w)
+    vis[w] = tree_tile ? vis_word(slot0 + 32 * w, g.P, g.N, row_valid, anc) : 0xffffffffu;
+  tmem_ld_wait();
+  if (tree_tile) {
+    // invisible keys become -inf: they drop out of the max and get P = 2^-inf = 0
+#pragma unroll
+    for (int c = 0; c < 64; ++c)
+      if (!((vis[c >> 5] >> (c & 31)) & 1u)) sr[c] = 0xff800000u;
+  }
+  float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 64; c += 8) {
+    a0 = fmax3(a0, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
+    a1 = fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+    a2 = fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+    a3 = fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+  }
+  return fmax3(a0, a1, fmaxf(a2, a3));
+}
+
+// P = 2^(s * scale - m) of 64 keys into their 32 bf16-pair columns at taddr_p; returns their sum.
+__device__ __forceinline__ float exp_store_half(uint32_t taddr_p, const uint32_t (&sr)[64], uint64_t sl2x2,
+                                                uint64_t nm2) {
+  uint64_t acc0 = 0, acc1 = 0;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+      const int cc = 32 * q + c;
+      const uint64_t y = f2_fma(f2_pack(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), sl2x2, nm2);
+      float y0, y1;
+      f2_unpack(y, y0, y1);
+      const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
+      if ((c >> 1) & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
+      else acc0 = f2_add(acc0, f2_pack(p0, p1));
+      pk[c >> 1] = pack_bf16x2_alu(p0, p1);
+    }
+    tmem_st16(taddr_p + 16 * q, pk);
+  }
+  float u0, u1, v0, v1;
+  f2_unpack(acc0, u0, u1);
+  f2_unpack(acc1, v0, v1);
+  return (u0 + u1) + (v0 + v1);
+}
+
+// The two softmax warpgroups take the kv tiles in turn (tile i of this CTA's sequence: warpgroup i % 2), each
+// thread owning one row, so that one warpgroup's exponentials overlap the other's loads and maximum.  The
+// online softmax's running maximum is decided tile by tile in order: the thread of tile i takes tile i - 1's
+// decision from shared memory (named barrier 2 + (i - 1) % 2: its owner arrives, this thread syncs), raises
+// it lazily (only by more than 2^8) with tile i's maximum, publishes it for tile i + 1, rescales O (after
+// PV of tile i - 1) when it was raised, and writes P relative to it.  Each thread keeps its own row sum
+// relative to the last maximum it saw; the two are merged at the segment's end.
+//
+// A warp whose wait gives up keeps running the loop structure with its work skipped (ok = false), so that the
+// named barriers the softmax threads share are always reached by all of them.
 __device__ bool softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uint32_t tmem, uint32_t rank) {
-  const int h = (static_cast<int>(threadIdx.x) - 128) >> 7;  // warpgroup: columns [64 h, 64 h + 64)
+  const int h = (static_cast<int>(threadIdx.x) - 128) >> 7;  // warpgroup
   const int r = threadIdx.x & 127;                             // row of this CTA's 128 == TMEM lane
   const int wq = (threadIdx.x >> 5) & 3;
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
@@ -614,6 +677,13 @@ __device__ bool softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
   const float sl2 = p.scale_log2;
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
   const int nodes_per_half = kBM / p.group;
+  // the CTA's last tile publishes no decision (no tile follows it)
+  uint32_t total = 0;
+  {
+    SegIter cnt = iter;
+    Seg gc;
+    while (cnt.next(s, p, gc)) total += static_cast<uint32_t>(gc.ke - gc.kb);
+  }
   bool ok = true;
   Seg g;
   uint32_t it = 0, sidx = 0;
@@ -624,101 +694,68 @@ __device__ bool softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
     const bool row_valid = node < g.N;
     if (static_cast<long long>(g.ke) * kBN > g.P && !build_ancestors(s, p, g)) ok = false;
     const uint32_t* anc = &s.anc[row_valid ? node : 0][0];
-    float m_use = -INFINITY, l = 0.f;
+    float m_cur = -INFINITY, l = 0.f;  // this thread's view of the running maximum, its row sum under it
+    bool did_last = false;
     for (int t = g.kb; t < g.ke; ++t, ++it) {
+      if (static_cast<int>(it & 1) != h) continue;  // the other warpgroup's tile
       const bool tree_tile = (t + 1) * kBN > g.P;
       const int sb = it % kSBufs;
-      const uint32_t s_col = sb * 128 + 64 * h;
+      const uint32_t s_addr = lane_base + sb * 128;
       if (ok && !warp_wait(&s.sfull[sb], (it / kSBufs) & 1, abort)) ok = false;
-      uint32_t sr[64];
-      float mloc = -INFINITY;
+      // pass 1: the tile's row maximum (raw scores)
+      float mraw = -INFINITY;
       if (ok) {
         tc_fence_after();
-        tmem_ld32(lane_base + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(lane_base + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        uint32_t vis[2];
-#pragma unroll
-        for (int w = 0; w < 2; ++w)
-          vis[w] = tree_tile ? vis_word(t * kBN + 64 * h + 32 * w, g.P, g.N, row_valid, anc) : 0xffffffffu;
-        tmem_ld_wait();
-        if (tree_tile) {
-          // invisible keys become -inf: they drop out of the max and get P = 2^-inf = 0
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (!((vis[c >> 5] >> (c & 31)) & 1u)) sr[c] = 0xff800000u;
-        }
-        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-          a0 = fmax3(a0, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
-          a1 = fmax3(a1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-          a2 = fmax3(a2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-          a3 = fmax3(a3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
-        }
-        mloc = fmax3(a0, a1, fmaxf(a2, a3));
+        uint32_t sr[64];
+        mraw = load_masked_half(s_addr, sr, tree_tile, t * kBN, g, row_valid, anc);
+        mraw = fmaxf(mraw, load_masked_half(s_addr + 64, sr, tree_tile, t * kBN + 64, g, row_valid, anc));
       }
-      // the row's maximum over both halves: the two threads of a row swap theirs (both have loaded S, so
-      // P may then be written over any of the row's S columns)
-      float* red = s.red[it & 1][0];
-      red[h * kBM + r] = mloc;
-      softmax_bar();
-      if (!ok) continue;
-      const float mraw = fmaxf(red[r], red[kBM + r]);
       const float mx = (mraw == -INFINITY) ? -INFINITY : mraw * sl2;
-      float alpha = 1.f;
-      bool resc = false;
-      if (mx > m_use + kRescaleThreshold) {
-        if (m_use != -INFINITY) {
-          alpha = ex2_approx(m_use - mx);
-          l *= alpha;
-          resc = (t > g.kb);
-        }
-        m_use = mx;
+      // the running maximum after the previous tile (its owner is the other warpgroup)
+      float m_prev = -INFINITY;
+      if (it > 0) {
+        named_bar_sync(2 + ((it - 1) & 1), kSoftmaxThreads);
+        if (t > g.kb) m_prev = s.mhand[(it - 1) & 1][r];
       }
+      const float m_new = (m_prev == -INFINITY || mx > m_prev + kRescaleThreshold) ? mx : m_prev;
+      if (it + 1 < total) {
+        s.mhand[it & 1][r] = m_new;
+        named_bar_arrive(2 + (it & 1), kSoftmaxThreads);
+      }
+      if (!ok) continue;
+      if (m_cur != m_new) {  // the other warpgroup (or this tile) raised the maximum: rescale this thread's sum
+        if (m_cur != -INFINITY) l *= ex2_approx(m_cur - m_new);
+        m_cur = m_new;
+      }
+      const bool resc = m_prev != -INFINITY && m_new != m_prev;
       if (__any_sync(0xffffffffu, resc)) {
-        // O holds PV of the segment's tiles so far; the last of them (tile it - 1) may still be running
+        // O holds PV of the segment's tiles so far, under m_prev; the last of them (tile it - 1) may still run
         if (!warp_wait(&s.pvdone[(it - 1) % kSBufs], ((it - 1) / kSBufs) & 1, abort)) {
           ok = false;
           continue;
         }
         tc_fence_after();
-        const float a = resc ? alpha : 1.f;
+        const float a = resc ? ex2_approx(m_prev - m_new) : 1.f;
 #pragma unroll
-        for (int cc = 0; cc < 64; cc += 32) {
+        for (int cc = 0; cc < 128; cc += 32) {
           uint32_t o[32];
-          tmem_ld32(lane_base + kTmO + 64 * h + cc, o);
+          tmem_ld32(lane_base + kTmO + cc, o);
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * a);
-          tmem_st32(lane_base + kTmO + 64 * h + cc, o);
+          tmem_st32(lane_base + kTmO + cc, o);
         }
       }
-      const float negm = (m_use == -INFINITY) ? 0.f : -m_use;
+      // pass 2: P over the keys of each half; keys [64 k, 64 k + 64) go to columns [32 k, 32 k + 32), over S
+      // columns this pass has already read
+      const float negm = (m_new == -INFINITY) ? 0.f : -m_new;
       const uint64_t nm2 = f2_pack(negm, negm);
-      // P = 2^(s * scale - m), row sum in packed pairs, bf16 pairs of P written over S: keys
-      // [64 h, 64 h + 64) go to columns [32 h, 32 h + 32) of the buffer, 16 columns at a time
-      uint64_t acc0 = 0, acc1 = 0;
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const int cc = 32 * q + c;
-          const uint64_t y = f2_fma(f2_pack(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), sl2x2, nm2);
-          float y0, y1;
-          f2_unpack(y, y0, y1);
-          const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
-          if ((c >> 1) & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
-          else acc0 = f2_add(acc0, f2_pack(p0, p1));
-          pk[c >> 1] = pack_bf16x2_alu(p0, p1);
-        }
-        tmem_st16(lane_base + sb * 128 + 32 * h + 16 * q, pk);
-      }
       {
-        float u0, u1, v0, v1;
-        f2_unpack(acc0, u0, u1);
-        f2_unpack(acc1, v0, v1);
-        l += (u0 + u1) + (v0 + v1);
+        uint32_t sr[64];
+        load_masked_half(s_addr, sr, tree_tile, t * kBN, g, row_valid, anc);
+        l += exp_store_half(s_addr, sr, sl2x2, nm2);
+        load_masked_half(s_addr + 64, sr, tree_tile, t * kBN + 64, g, row_valid, anc);
+        l += exp_store_half(s_addr + 32, sr, sl2x2, nm2);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -727,22 +764,28 @@ __device__ bool softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
         if (rank == 0) mbar_arrive(&s.pfull[sb]);
         else mbar_arrive_cluster_relaxed(pfull0 + sb * 8);
       }
+      did_last = (t == g.ke - 1);
     }
     // ---------------- epilogue of the segment
     bool seg_ok = false;
     if (ok && !warp_wait(&s.metafull[buf], (sidx >> 1) & 1, abort)) ok = false;
-    if (ok) {
-      seg_ok = s.meta_valid[buf] != 0;
-      if (!warp_wait(&s.pvdone[(it - 1) % kSBufs], ((it - 1) / kSBufs) & 1, abort)) ok = false;  // last PV
+    if (ok) seg_ok = s.meta_valid[buf] != 0;
+    // The warpgroup of the segment's last tile waits for its PV (every earlier MMA is complete then too); the
+    // barrier below tells the other warpgroup.
+    if (ok && did_last && !warp_wait(&s.pvdone[(it - 1) % kSBufs], ((it - 1) / kSBufs) & 1, abort)) ok = false;
+    s.lsum[buf][h][r] = l;
+    s.msum[buf][h][r] = m_cur;
+    softmax_bar();
+    float l_tot = 0.f, m_fin = -INFINITY;
+    {
+      const float m0 = s.msum[buf][0][r], m1 = s.msum[buf][1][r];
+      m_fin = fmaxf(m0, m1);
+      if (m0 != -INFINITY) l_tot += s.lsum[buf][0][r] * ex2_approx(m0 - m_fin);
+      if (m1 != -INFINITY) l_tot += s.lsum[buf][1][r] * ex2_approx(m1 - m_fin);
     }
     if (ok) {
       tc_fence_after();
       mbar_arrive(&s.metaempty[buf]);
-    }
-    s.lsum[h][r] = l;
-    softmax_bar();
-    const float l_tot = s.lsum[0][r] + s.lsum[1][r];
-    if (ok) {
       const bool split = g.c0 != g.c1;
       const long long grow = static_cast<long long>(g.off + node) * p.hq + head;  // global row
       if (!split) {
@@ -755,7 +798,7 @@ __device__ bool softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
           if (seg_ok && row_valid) store_half_row_bf16(p.out + grow * 128 + 64 * h + cc, o, inv_l);
         }
         if (seg_ok && row_valid && h == 0 && p.lse != nullptr)
-          p.lse[grow] = (m_use + __log2f(l_tot)) * 0.69314718055994531f;
+          p.lse[grow] = (m_fin + __log2f(l_tot)) * 0.69314718055994531f;
       } else {
         // unit cut between pairs: store this segment's unnormalised O, (m, l) and validity; the combine
         // kernel that runs after this one merges the segments
@@ -772,7 +815,7 @@ __device__ bool softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
                                __uint_as_float(o[c + 3])));
         }
         if (h == 0) {
-          __stcg(&p.part_ml[static_cast<long long>(myslot) * kBM + r], make_float2(m_use, l_tot));
+          __stcg(&p.part_ml[static_cast<long long>(myslot) * kBM + r], make_float2(m_fin, l_tot));
           __stcg(&p.part_ok[static_cast<long long>(myslot) * kBM + r], seg_ok ? 1 : 0);
         }
         if (iter.pair == g.c0 && rank == 0 && h == 0 && r == 0) {
