@@ -1,8 +1,7 @@
-"""Host-side model of the attention kernel's stream-K partition over CTA pairs (the same integer formulas as
-the device plan; a unit is one 256-row M tile of one (sequence, kv head), a "cta" below is one CTA pair):
-every (unit, kv tile) pair is covered exactly once, a unit's sharing pairs are exactly those that hold one of
-its kv tiles, partial slots never collide, every pair's range is non-empty, and a pair that starts segments
-in mid-range gets correspondingly fewer kv tiles.
+"""Host-side model of the attention kernel's stream-K partition (the same integer formulas as the
+device plan): every (unit, kv tile) pair is covered exactly once, a unit's sharing CTAs are exactly
+those that hold one of its kv tiles, partial slots never collide, every CTA's range is non-empty, and
+a CTA that starts segments in mid-range gets correspondingly fewer kv tiles.
 
 Each unit costs SEG_COST + kt positions: SEG_COST leading positions (the price of starting a segment
 in mid-kernel) and then its kt kv tiles."""
@@ -10,7 +9,7 @@ in mid-kernel) and then its kt kv tiles."""
 import numpy as np
 import pytest
 
-BN, BM = 128, 256  # keys per kv tile, rows per M tile (a CTA pair's)
+BN, BM = 128, 128
 SEG_COST = 3
 
 
@@ -59,13 +58,12 @@ def segments(prefix, nodes, hkv, group, grid):
 
 
 @pytest.mark.parametrize("prefix,nodes,hkv,group,grid", [
-    ([256], [16], 1, 4, 74),
-    ([4096], [256], 8, 4, 74),
-    ([32768] * 4, [256] * 4, 4, 8, 74),
-    (list(np.random.default_rng(0).integers(1024, 8193, 16)), [64] * 16, 8, 4, 74),
+    ([256], [16], 1, 4, 148),
+    ([4096], [256], 8, 4, 148),
+    ([32768] * 4, [256] * 4, 4, 8, 148),
+    (list(np.random.default_rng(0).integers(1024, 8193, 16)), [64] * 16, 8, 4, 148),
     ([0, 5, 300, 17], [3, 0, 256, 1], 2, 2, 7),
-    ([10] * 50, [1] * 50, 1, 1, 74),
-    ([4096], [200], 2, 16, 74),
+    ([10] * 50, [1] * 50, 1, 1, 148),
 ])
 def test_cover_exactly_once(prefix, nodes, hkv, group, grid):
     segs, W, G = segments(prefix, nodes, hkv, group, grid)

@@ -27,6 +27,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+int sm_count() {
+  static std::atomic<int> counts[jf::kMaxDevices];
+  const int dev = jf::current_device();
+  if (dev < 0) return -1;
+  int n = counts[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    counts[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // 3-D bf16 tensor map, dims innermost first, 128-byte swizzle, out-of-range boxes read as zero.
@@ -93,6 +105,10 @@ jf_status jf_tree_attention(const void* q, const void* k_cache, const void* v_ca
     return JF_ERR_INVALID_ARG;
   if (workspace_bytes < AttnWorkspace::total) return JF_ERR_INVALID_ARG;
 
+  const int sms = sm_count();
+  if (sms <= 0) return JF_ERR_CUDA;
+  const int grid = sms < kMaxGrid ? sms : kMaxGrid;
+
   CUtensorMap tm_q, tm_k, tm_v;
   const uint64_t row = kHeadDim * sizeof(__nv_bfloat16);  // 256 bytes
   if (!encode_3d(&tm_q, q, kHeadDim, num_q_heads, total_nodes, row, row * num_q_heads, 64, group,
@@ -125,7 +141,7 @@ jf_status jf_tree_attention(const void* q, const void* k_cache, const void* v_ca
   p.max_pages = max_pages_per_seq;
   p.num_pages = num_pages;
   p.scale_log2 = sm_scale * 1.4426950408889634f;
-  if (launch_tree_attention(tm_q, tm_k, tm_v, p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (launch_tree_attention(tm_q, tm_k, tm_v, p, grid, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return JF_ERR_CUDA;
   return JF_OK;
 }

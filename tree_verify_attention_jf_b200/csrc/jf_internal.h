@@ -48,9 +48,9 @@ constexpr int kPageSize = 16;
 constexpr int kMaxTreeNodes = 256;          // nodes per sequence in jf_tree_attention
 constexpr int kAncWords = kMaxTreeNodes / 32;
 constexpr int kMaxAttnBatch = 1024;
-constexpr int kMaxGrid = 256;               // persistent CTA pairs (one CTA per SM, capped)
-constexpr int kAttnRows = 128;              // rows of an M tile held by one CTA of a pair
-constexpr int kAttnQTiles = 2;              // CTAs (row halves) per M tile
+constexpr int kMaxGrid = 256;               // persistent CTAs (one per SM, capped)
+constexpr int kAttnRows = 128;              // rows of one M tile
+constexpr int kAttnQTiles = 2;              // M tiles per work unit (they share every K/V tile)
 
 struct AttnParams {
   const int32_t* block_table;
@@ -62,8 +62,7 @@ struct AttnParams {
   float* part_o;    // [2*kMaxGrid*2][32][128] float4 partial outputs (slot, column quad, row)
   float2* part_ml;  // [2*kMaxGrid*2][128] (running max in log2 units, row sum)
   int32_t* part_ok; // [2*kMaxGrid*2][128] 1 = the partial's sequence passed its device checks
-  int4* units;      // [kMaxGrid] descriptor of the split unit whose first CTA pair is i (last pair, first node,
-                    // nodes, kv head)
+  int4* units;      // [kMaxGrid] descriptor of the split unit whose first CTA is i (c1, first node, nodes, kv head)
   int32_t* status;
   int batch, total_nodes, hq, hkv, group, max_pages, num_pages;
   float scale_log2;
@@ -71,7 +70,7 @@ struct AttnParams {
 
 // Workspace layout of jf_tree_attention (offsets in bytes, each 256-aligned).
 struct AttnWorkspace {
-  static constexpr size_t kSlots = 2 * kMaxGrid * kAttnQTiles;  // (CTA pair, first/last segment, row half)
+  static constexpr size_t kSlots = 2 * kMaxGrid * kAttnQTiles;  // (CTA, first/last segment, Q tile)
   static constexpr size_t units_off = 0;
   static constexpr size_t units_bytes = sizeof(int4) * kMaxGrid;
   static constexpr size_t ok_off = units_off + ((units_bytes + 255) & ~size_t(255));
@@ -85,7 +84,7 @@ struct AttnWorkspace {
 
 size_t attention_smem_bytes();
 cudaError_t launch_tree_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                                  const AttnParams& p, cudaStream_t stream);
+                                  const AttnParams& p, int grid, cudaStream_t stream);
 
 // ---- tree build
 constexpr int kMaxTopk = 8;
