@@ -341,8 +341,12 @@ def graph_timer(args, stream, flush):
     return capture, timed
 
 
-def attention_leg(name, args, device, capture, timed, pk):
-    """Tree attention alone on one of the seeded attention workloads (the inputs the parity tests use)."""
+FP8_SCALES = (1.0 / 128, 1.0 / 64)  # K and V cache scales of the 8-bit legs (N(0, 0.5) values -> codes in +-448)
+
+
+def attention_leg(name, args, device, capture, timed, pk, fp8=False):
+    """Tree attention alone on one of the seeded attention workloads (the inputs the parity tests use); with
+    fp8, over the same cache stored as 8-bit E4M3 codes (jf_tree_attention_fp8)."""
     import torch
 
     from tree_verify_attention_jf_b200 import api, synth, workloads
@@ -350,13 +354,22 @@ def attention_leg(name, args, device, capture, timed, pk):
     inp = workloads.attention_workload(name)
     bf = lambda a: synth.to_bf16_tensor(a).to(device)
     i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
-    q, kc, vc = bf(inp.q), bf(inp.k_cache), bf(inp.v_cache)
+    q = bf(inp.q)
+    if fp8:
+        kc = torch.from_numpy(synth.e4m3_cache(inp.k_cache, FP8_SCALES[0])).to(device)
+        vc = torch.from_numpy(synth.e4m3_cache(inp.v_cache, FP8_SCALES[1])).to(device)
+    else:
+        kc, vc = bf(inp.k_cache), bf(inp.v_cache)
     bt, pl, offs, par = i32(inp.block_table), i32(inp.prefix_lens), i32(inp.tree_offsets), i32(inp.parent)
     out = torch.empty_like(q)
     ws = api.AttentionWorkspace(torch.device(device))
 
     def call():
-        api.tree_attention(q, kc, vc, bt, pl, offs, par, inp.sm_scale, out=out, workspace=ws)
+        if fp8:
+            api.tree_attention_fp8(q, kc, vc, FP8_SCALES[0], FP8_SCALES[1], bt, pl, offs, par, inp.sm_scale, out=out,
+                                   workspace=ws)
+        else:
+            api.tree_attention(q, kc, vc, bt, pl, offs, par, inp.sm_scale, out=out, workspace=ws)
 
     call()
     torch.cuda.synchronize()
@@ -368,13 +381,18 @@ def attention_leg(name, args, device, capture, timed, pk):
     prefix = [int(x) for x in inp.prefix_lens]
     pairs = visible_pairs_ragged(inp.parent, offs_h, prefix)
     flops, nbytes = attention_work(nodes, inp.num_q_heads, inp.num_kv_heads, prefix, pairs)
+    if fp8:  # the cache's bytes are halved (one byte per element)
+        nbytes -= sum(inp.num_kv_heads * (P + n) * HEAD_DIM * 2 for P, n in zip(prefix, nodes))
     tflops = flops / (ms * 1e-3) / 1e12
     gbs = nbytes / (ms * 1e-3) / 1e9
-    leg = {"call": "jf_tree_attention", "ms": ms, "nodes": sum(nodes), "nodes_per_s": sum(nodes) / (ms * 1e-3),
+    leg = {"call": "jf_tree_attention_fp8" if fp8 else "jf_tree_attention", "ms": ms, "nodes": sum(nodes), "nodes_per_s": sum(nodes) / (ms * 1e-3),
            "batch": inp.batch, "q_heads": inp.num_q_heads, "kv_heads": inp.num_kv_heads,
            "prefix": prefix if len(prefix) <= 4 else f"{min(prefix)}..{max(prefix)} (mean {statistics.mean(prefix):.0f})",
            "algorithmic_flops": flops, "algorithmic_bytes": nbytes, "tflops": tflops, "gbs": gbs,
-           "tensor_frac": tflops / pk["bf16"], "hbm_frac": gbs / pk["hbm"], "traffic": attention_traffic(name)}
+           "tensor_frac": tflops / pk["bf16"], "hbm_frac": gbs / pk["hbm"],
+           "traffic": attention_traffic(name + ("_fp8" if fp8 else ""))}
+    if fp8:
+        leg["cache"] = f"E4M3 codes, k_scale {FP8_SCALES[0]}, v_scale {FP8_SCALES[1]}"
     if name in HBM_BOUND:
         leg.update(bound="hbm", frac=gbs / pk["hbm"])
     elif name == "tiny":
@@ -641,6 +659,9 @@ def run_gpu(args, cfg, rank, world, device):
             if name != args.workload:
                 legs[name] = attention_leg(name, args, device, capture, timed, pk)
                 torch.cuda.empty_cache()
+        # the serving batch over an 8-bit (E4M3) cache: half the cache bytes
+        legs["serving_fp8"] = attention_leg("serving", args, device, capture, timed, pk, fp8=True)
+        torch.cuda.empty_cache()
         legs.update(build_accept_leg(args, device, capture, timed, pk))
         torch.cuda.empty_cache()
         legs["expand_frontier"] = frontier_leg(args, device, flush, pk)

@@ -109,6 +109,31 @@ JF_API jf_status jf_tree_attention(const void* q, const void* k_cache, const voi
                             size_t workspace_bytes, int32_t* dev_status, jf_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * jf_tree_attention_fp8 -- jf_tree_attention over a paged KV cache stored in 8 bits (E4M3).
+ *
+ * The attention of jf_tree_attention [JF section 2 tree-causal mask; section 3 paged attention in the
+ * serving engine] over the decoded cache: a stored code c stands for decode(c) * k_scale in k_cache
+ * and decode(c) * v_scale in v_cache, where decode is the E4M3 format (1 sign, 4 exponent bits with
+ * bias 7, 3 mantissa bits, no infinities; S.1111.111 is NaN; largest magnitude 448).  The pages do not
+ * describe 8-bit caches; this is the serving variant for heavy load, where the cache's bytes dominate.
+ * The result is the bf16 path's definition applied to the decoded values: the kernel computes on the
+ * exact decoded values (every E4M3 value is exact in f16) with q converted to f16, applies k_scale in
+ * the softmax scale and v_scale in the final normalisation; tolerances as for jf_tree_attention.
+ *
+ * Layouts: as jf_tree_attention except k_cache, v_cache: uint8 E4M3 codes [num_pages, page_size,
+ * num_kv_heads, head_dim], 16-byte aligned.  k_scale, v_scale: finite and > 0.  q stays bf16
+ * (values beyond the f16 range, |q| > 65504, are not supported).  Same workspace, limits, device
+ * checks and errors as jf_tree_attention.
+ * ------------------------------------------------------------------------------------------ */
+JF_API jf_status jf_tree_attention_fp8(const void* q, const void* k_cache, const void* v_cache, float k_scale,
+                                       float v_scale, const int32_t* block_table, int max_pages_per_seq,
+                                       const int32_t* prefix_lens, const int32_t* tree_offsets,
+                                       const int32_t* parent, int batch, int total_nodes, int num_q_heads,
+                                       int num_kv_heads, int head_dim, int page_size, int num_pages,
+                                       float sm_scale, void* out, float* lse, void* workspace,
+                                       size_t workspace_bytes, int32_t* dev_status, jf_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * jf_build_tree -- best-first draft-tree construction under a token budget.
  *
  * Defines [JF section 2, "tree construction": the head emits logits for all depths in parallel; the

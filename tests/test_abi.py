@@ -18,7 +18,7 @@ def test_exports_every_declared_symbol(L):
     assert set(names) == {"jf_status_string", "jf_version", "jf_tree_attention_workspace_size", "jf_tree_attention",
                           "jf_build_tree_workspace_size", "jf_build_tree", "jf_build_tree_noalloc", "jf_accept",
                           "jf_commit_kv", "jf_tree_kv_append", "jf_expand_frontier_state_size",
-                          "jf_expand_frontier_workspace_size", "jf_expand_frontier"}
+                          "jf_expand_frontier_workspace_size", "jf_expand_frontier", "jf_tree_attention_fp8"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -157,3 +157,19 @@ def test_expand_frontier_host_validation(L):
         assert call(**bad) == _lib.JF_ERR_INVALID_ARG, bad
     assert L.jf_expand_frontier_state_size(2, 64, 4) >= 2 * 64 * (8 + 4 * 8 + 4 * 4 + 4)
     assert L.jf_expand_frontier_workspace_size(2, 4, 4096) == 2 * 4 * 1 * 80
+
+
+def test_tree_attention_fp8_host_validation(L):
+    def call(**over):
+        a = dict(ks=0.01, vs=0.02, batch=1, T=16, hq=4, hkv=1, d=128, page=16, pages=8, scale=0.088)
+        a.update(over)
+        return L.jf_tree_attention_fp8(None, None, None, a["ks"], a["vs"], None, 4, None, None, None, a["batch"],
+                                       a["T"], a["hq"], a["hkv"], a["d"], a["page"], a["pages"], a["scale"], None, None,
+                                       None, 0, None, None)
+    assert call() == _lib.JF_ERR_INVALID_ARG  # null pointers
+    for bad in (dict(ks=0.0), dict(vs=-1.0), dict(ks=float("inf")), dict(vs=float("nan")), dict(scale=0.0)):
+        assert call(**bad) == _lib.JF_ERR_INVALID_ARG, bad
+    assert call(d=64) == _lib.JF_ERR_UNSUPPORTED
+    assert call(page=32) == _lib.JF_ERR_UNSUPPORTED
+    assert call(hq=6, hkv=4) == _lib.JF_ERR_UNSUPPORTED
+    assert call(batch=0) == _lib.JF_OK

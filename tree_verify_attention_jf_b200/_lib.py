@@ -45,6 +45,9 @@ def lib() -> ctypes.CDLL:
     L.jf_tree_attention_workspace_size.restype = sz
     L.jf_tree_attention.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp, sz, vp, vp]
     L.jf_tree_attention.restype = i
+    L.jf_tree_attention_fp8.argtypes = [vp, vp, vp, f, f, vp, i, vp, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp, sz,
+                                        vp, vp]
+    L.jf_tree_attention_fp8.restype = i
     L.jf_build_tree_workspace_size.argtypes = [i, i, i, i]
     L.jf_build_tree_workspace_size.restype = sz
     L.jf_build_tree.argtypes = [vp, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, sz, vp, vp]

@@ -79,6 +79,41 @@ def tree_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     return out
 
 
+def tree_attention_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k_scale: float,
+                       v_scale: float, block_table: torch.Tensor, prefix_lens: torch.Tensor, tree_offsets: torch.Tensor,
+                       parent: torch.Tensor, sm_scale: float, out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None, workspace: Optional[AttentionWorkspace] = None,
+                       dev_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """jf_tree_attention_fp8: as :func:`tree_attention`, with k/v_cache uint8 E4M3 codes [pages, 16, Hkv, 128]
+    standing for decode(code) * k_scale / v_scale.  Returns out (bf16)."""
+    dev = q.device
+    T, Hq, D = q.shape
+    num_pages, page, Hkv, D2 = k_cache.shape
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.uint8, dev)
+    _need(v_cache, "v_cache", torch.uint8, dev)
+    for name, t in (("block_table", block_table), ("prefix_lens", prefix_lens), ("tree_offsets", tree_offsets),
+                    ("parent", parent)):
+        _need(t, name, torch.int32, dev)
+    if v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache shapes differ")
+    B = prefix_lens.numel()
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev)
+    if workspace is None:
+        workspace = AttentionWorkspace(dev)
+    code = _lib.lib().jf_tree_attention_fp8(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale), _ptr(block_table),
+        block_table.shape[1] if block_table.dim() == 2 else 0, _ptr(prefix_lens), _ptr(tree_offsets), _ptr(parent), B,
+        T, Hq, Hkv, D, page, num_pages, float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace.buf), workspace.nbytes,
+        _ptr(dev_status), _stream(stream))
+    _lib.check("jf_tree_attention_fp8", code)
+    return out
+
+
 def build_tree_workspace(batch: int, depths: int, vocab: int, topk: int, device) -> torch.Tensor:
     n = _lib.lib().jf_build_tree_workspace_size(batch, depths, vocab, topk)
     return torch.empty(max(n, 16), dtype=torch.uint8, device=device)

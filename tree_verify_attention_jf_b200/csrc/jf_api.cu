@@ -41,18 +41,100 @@ int sm_count() {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// 3-D bf16 tensor map, dims innermost first, 128-byte swizzle, out-of-range boxes read as zero.
+// 3-D tensor map, dims innermost first, out-of-range boxes read as zero: bf16 with 128-byte swizzle, or
+// 8-bit elements (E4M3 codes) with no swizzle.
 bool encode_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
-               uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2) {
+               uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2, bool bytes = false) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
   const cuuint32_t box[3] = {b0, b1, b2};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            bytes ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// jf_tree_attention and jf_tree_attention_fp8: validation, tensor maps, workspace carving, launch.
+jf_status tree_attention_call(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                              int max_pages_per_seq, const int32_t* prefix_lens, const int32_t* tree_offsets,
+                              const int32_t* parent, int batch, int total_nodes, int num_q_heads, int num_kv_heads,
+                              int head_dim, int page_size, int num_pages, float sm_scale, bool fp8, float k_scale,
+                              float v_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                              int32_t* dev_status, jf_stream_t stream) {
+  using namespace jf;
+  if (batch < 0 || total_nodes < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_pages_per_seq <= 0 ||
+      num_pages <= 0)
+    return JF_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return JF_ERR_INVALID_ARG;
+  if (!(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale))
+    return JF_ERR_INVALID_ARG;
+  if (!std::isfinite(sm_scale * k_scale)) return JF_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || page_size != kPageSize) return JF_ERR_UNSUPPORTED;
+  if (num_q_heads % num_kv_heads != 0) return JF_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8 && group != 16) return JF_ERR_UNSUPPORTED;
+  if (batch > kMaxAttnBatch) return JF_ERR_UNSUPPORTED;
+  if (static_cast<long long>(num_pages) * kPageSize >= (1ll << 31)) return JF_ERR_UNSUPPORTED;
+  if (batch == 0 || total_nodes == 0) return JF_OK;
+  if (!q || !k_cache || !v_cache || !block_table || !prefix_lens || !tree_offsets || !parent || !out || !workspace)
+    return JF_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(workspace, 256))
+    return JF_ERR_INVALID_ARG;
+  if (workspace_bytes < AttnWorkspace::total) return JF_ERR_INVALID_ARG;
+
+  const int sms = sm_count();
+  if (sms <= 0) return JF_ERR_CUDA;
+  const int grid = sms < kMaxGrid ? sms : kMaxGrid;
+
+  CUtensorMap tm_q, tm_k, tm_v;
+  const uint64_t row = kHeadDim * sizeof(__nv_bfloat16);  // 256 bytes
+  if (!encode_3d(&tm_q, q, kHeadDim, num_q_heads, total_nodes, row, row * num_q_heads, 64, group,
+                 kAttnRows / group))
+    return JF_ERR_CUDA;
+  const uint64_t slots = static_cast<uint64_t>(num_pages) * kPageSize;
+  if (fp8) {  // one byte per element: whole 128-byte rows, 16 slots a box
+    if (!encode_3d(&tm_k, k_cache, kHeadDim, num_kv_heads, slots, kHeadDim, kHeadDim * num_kv_heads, kHeadDim, 1,
+                   kPageSize, true))
+      return JF_ERR_CUDA;
+    if (!encode_3d(&tm_v, v_cache, kHeadDim, num_kv_heads, slots, kHeadDim, kHeadDim * num_kv_heads, kHeadDim, 1,
+                   kPageSize, true))
+      return JF_ERR_CUDA;
+  } else {
+    if (!encode_3d(&tm_k, k_cache, kHeadDim, num_kv_heads, slots, row, row * num_kv_heads, 64, 1, kPageSize))
+      return JF_ERR_CUDA;
+    if (!encode_3d(&tm_v, v_cache, kHeadDim, num_kv_heads, slots, row, row * num_kv_heads, 64, 1, kPageSize))
+      return JF_ERR_CUDA;
+  }
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  AttnParams p;
+  p.block_table = block_table;
+  p.prefix_lens = prefix_lens;
+  p.tree_offsets = tree_offsets;
+  p.parent = parent;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.units = reinterpret_cast<int4*>(ws + AttnWorkspace::units_off);
+  p.part_ok = reinterpret_cast<int32_t*>(ws + AttnWorkspace::ok_off);
+  p.part_ml = reinterpret_cast<float2*>(ws + AttnWorkspace::ml_off);
+  p.part_o = reinterpret_cast<float*>(ws + AttnWorkspace::o_off);
+  p.status = dev_status;
+  p.batch = batch;
+  p.total_nodes = total_nodes;
+  p.hq = num_q_heads;
+  p.hkv = num_kv_heads;
+  p.group = group;
+  p.max_pages = max_pages_per_seq;
+  p.num_pages = num_pages;
+  p.scale_log2 = sm_scale * k_scale * 1.4426950408889634f;
+  p.v_scale = v_scale;
+  if (launch_tree_attention(tm_q, tm_k, tm_v, p, grid, fp8, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JF_ERR_CUDA;
+  return JF_OK;
 }
 
 }  // namespace
@@ -86,64 +168,20 @@ jf_status jf_tree_attention(const void* q, const void* k_cache, const void* v_ca
                             const int32_t* parent, int batch, int total_nodes, int num_q_heads, int num_kv_heads,
                             int head_dim, int page_size, int num_pages, float sm_scale, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, int32_t* dev_status, jf_stream_t stream) {
-  using namespace jf;
-  if (batch < 0 || total_nodes < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_pages_per_seq <= 0 ||
-      num_pages <= 0)
-    return JF_ERR_INVALID_ARG;
-  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return JF_ERR_INVALID_ARG;
-  if (head_dim != kHeadDim || page_size != kPageSize) return JF_ERR_UNSUPPORTED;
-  if (num_q_heads % num_kv_heads != 0) return JF_ERR_UNSUPPORTED;
-  const int group = num_q_heads / num_kv_heads;
-  if (group != 1 && group != 2 && group != 4 && group != 8 && group != 16) return JF_ERR_UNSUPPORTED;
-  if (batch > kMaxAttnBatch) return JF_ERR_UNSUPPORTED;
-  if (static_cast<long long>(num_pages) * kPageSize >= (1ll << 31)) return JF_ERR_UNSUPPORTED;
-  if (batch == 0 || total_nodes == 0) return JF_OK;
-  if (!q || !k_cache || !v_cache || !block_table || !prefix_lens || !tree_offsets || !parent || !out || !workspace)
-    return JF_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
-      !aligned(workspace, 256))
-    return JF_ERR_INVALID_ARG;
-  if (workspace_bytes < AttnWorkspace::total) return JF_ERR_INVALID_ARG;
+  return tree_attention_call(q, k_cache, v_cache, block_table, max_pages_per_seq, prefix_lens, tree_offsets, parent,
+                             batch, total_nodes, num_q_heads, num_kv_heads, head_dim, page_size, num_pages, sm_scale,
+                             false, 1.f, 1.f, out, lse, workspace, workspace_bytes, dev_status, stream);
+}
 
-  const int sms = sm_count();
-  if (sms <= 0) return JF_ERR_CUDA;
-  const int grid = sms < kMaxGrid ? sms : kMaxGrid;
-
-  CUtensorMap tm_q, tm_k, tm_v;
-  const uint64_t row = kHeadDim * sizeof(__nv_bfloat16);  // 256 bytes
-  if (!encode_3d(&tm_q, q, kHeadDim, num_q_heads, total_nodes, row, row * num_q_heads, 64, group,
-                 kAttnRows / group))
-    return JF_ERR_CUDA;
-  const uint64_t slots = static_cast<uint64_t>(num_pages) * kPageSize;
-  if (!encode_3d(&tm_k, k_cache, kHeadDim, num_kv_heads, slots, row, row * num_kv_heads, 64, 1, kPageSize))
-    return JF_ERR_CUDA;
-  if (!encode_3d(&tm_v, v_cache, kHeadDim, num_kv_heads, slots, row, row * num_kv_heads, 64, 1, kPageSize))
-    return JF_ERR_CUDA;
-
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  AttnParams p;
-  p.block_table = block_table;
-  p.prefix_lens = prefix_lens;
-  p.tree_offsets = tree_offsets;
-  p.parent = parent;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  p.units = reinterpret_cast<int4*>(ws + AttnWorkspace::units_off);
-  p.part_ok = reinterpret_cast<int32_t*>(ws + AttnWorkspace::ok_off);
-  p.part_ml = reinterpret_cast<float2*>(ws + AttnWorkspace::ml_off);
-  p.part_o = reinterpret_cast<float*>(ws + AttnWorkspace::o_off);
-  p.status = dev_status;
-  p.batch = batch;
-  p.total_nodes = total_nodes;
-  p.hq = num_q_heads;
-  p.hkv = num_kv_heads;
-  p.group = group;
-  p.max_pages = max_pages_per_seq;
-  p.num_pages = num_pages;
-  p.scale_log2 = sm_scale * 1.4426950408889634f;
-  if (launch_tree_attention(tm_q, tm_k, tm_v, p, grid, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return JF_ERR_CUDA;
-  return JF_OK;
+jf_status jf_tree_attention_fp8(const void* q, const void* k_cache, const void* v_cache, float k_scale,
+                                float v_scale, const int32_t* block_table, int max_pages_per_seq,
+                                const int32_t* prefix_lens, const int32_t* tree_offsets, const int32_t* parent,
+                                int batch, int total_nodes, int num_q_heads, int num_kv_heads, int head_dim,
+                                int page_size, int num_pages, float sm_scale, void* out, float* lse, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, jf_stream_t stream) {
+  return tree_attention_call(q, k_cache, v_cache, block_table, max_pages_per_seq, prefix_lens, tree_offsets, parent,
+                             batch, total_nodes, num_q_heads, num_kv_heads, head_dim, page_size, num_pages, sm_scale,
+                             true, k_scale, v_scale, out, lse, workspace, workspace_bytes, dev_status, stream);
 }
 
 size_t jf_build_tree_workspace_size(int batch, int depths, int vocab, int topk) {

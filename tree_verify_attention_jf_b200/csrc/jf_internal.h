@@ -65,7 +65,8 @@ struct AttnParams {
   int4* units;      // [kMaxGrid] descriptor of the split unit whose first CTA is i (c1, first node, nodes, kv head)
   int32_t* status;
   int batch, total_nodes, hq, hkv, group, max_pages, num_pages;
-  float scale_log2;
+  float scale_log2;  // softmax scale (times the K cache's scale for an 8-bit cache) times log2(e)
+  float v_scale;     // the V cache's scale (1 for a bf16 cache)
 };
 
 // Workspace layout of jf_tree_attention (offsets in bytes, each 256-aligned).
@@ -83,8 +84,9 @@ struct AttnWorkspace {
 };
 
 size_t attention_smem_bytes();
+// fp8_cache: tm_k / tm_v describe 8-bit (E4M3) caches with whole 128-byte rows per box, no swizzle
 cudaError_t launch_tree_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                                  const AttnParams& p, int grid, cudaStream_t stream);
+                                  const AttnParams& p, int grid, bool fp8_cache, cudaStream_t stream);
 
 // ---- tree build
 constexpr int kMaxTopk = 8;

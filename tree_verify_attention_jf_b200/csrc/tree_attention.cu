@@ -27,6 +27,9 @@
 //     in a descriptor slot; combine_kernel, launched right behind on the
 //     same stream with a programmatic dependency, merges each recorded unit's partials and stores the
 //     bf16 output.  Nothing spins on another CTA.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "jf_device.cuh"
 #include "jf_internal.h"
 
@@ -59,6 +62,8 @@ struct __align__(1024) Smem {
   long long scan_warp[kThreads / 32];
   uint64_t bar_qfull, bar_qempty;
   uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
+  // 8-bit cache: the copies land on these; the copy warp converts the tile and then arrives on the full barrier
+  uint64_t bar_qland, bar_kland[kStages], bar_vland[kStages];
   uint64_t bar_sfull[kAttnQTiles], bar_pfull[kAttnQTiles], bar_pvdone[kAttnQTiles];
   uint64_t bar_metafull[2], bar_metaempty[2];
   uint32_t tmem_base;
@@ -186,16 +191,83 @@ __device__ void build_plan(Smem& s, const AttnParams& p) {
 }
 
 // ------------------------------------------------------------------------------------------------
-// Warps 0 and 2: K / V gathers (warp 0 also loads the Q tiles)
+// 8-bit (E4M3) cache: conversion to f16 in shared memory.  Every E4M3 value is exactly an f16, so the MMAs
+// run on f16 operands (Q converted from bf16, which it also represents exactly in the range of attention
+// inputs) and see exactly the decoded cache; the caches' scales are applied outside (K's in the softmax
+// scale, V's in the normalisation).
 // ------------------------------------------------------------------------------------------------
+// One K or V stage: the copy put the tile's 8-bit rows (128 keys x 128 dims, one 128-byte row per key) in the
+// stage's upper 16 KB; they become f16 in the 128-byte-swizzled [half][128 keys][64 dims] layout of the whole
+// stage.  A warp converts four rows per step: all lanes read their 16 bytes first, then write 2 x 16 bytes;
+// the writes of a step land in rows [0, 16 KB) and on the 8-bit rows the same step has just read, so rows
+// still to be read are never overwritten.
+__device__ __forceinline__ void convert_stage_e4m3(uint8_t* stage, int lane) {
+  const int c = lane & 7;  // 16-byte chunk of the 8-bit row: dims [16 c, 16 c + 16)
+  for (int r0 = 0; r0 < kBN; r0 += 4) {
+    const int row = r0 + (lane >> 3);
+    const uint4 raw = *reinterpret_cast<const uint4*>(stage + kHalfBytes + row * 128 + c * 16);
+    __syncwarp();
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t hv[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xffffu), __NV_E4M3);
+      const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
+      hv[2 * i] = static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16);
+      hv[2 * i + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
+    }
+    // dims [16 c, 16 c + 16) are f16 bytes [32 (c % 4), 32 (c % 4) + 32) of half c / 4: chunks 2 (c % 4) and + 1
+    const int j0 = 2 * (c & 3);
+    uint8_t* base = stage + (c >> 2) * kHalfBytes + row * 128;
+    *reinterpret_cast<uint4*>(base + ((j0 ^ (row & 7)) * 16)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    *reinterpret_cast<uint4*>(base + (((j0 + 1) ^ (row & 7)) * 16)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+    __syncwarp();
+  }
+}
+
+// The Q tiles in place, bf16 -> f16, element by element (the swizzle does not matter).
+__device__ __forceinline__ void convert_q_bf16_f16(uint8_t* q, int bytes, int lane) {
+  for (int i = lane * 16; i < bytes; i += 32 * 16) {
+    uint4 v = *reinterpret_cast<const uint4*>(q + i);
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const __half2 h = __floats2half2_rn(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
+      w[k] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(q + i) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Warps 0 and 2: K / V gathers (warp 0 also loads the Q tiles).  With an 8-bit cache each tile lands on a
+// barrier of its own; the warp converts it after issuing the next tile's copies and then arrives on the
+// full barrier the MMA warp waits on (the Q tiles likewise, after the segment's first K tile).
+// ------------------------------------------------------------------------------------------------
+template <bool kFp8>
 __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_v, const CUtensorMap* tm_q,
                             const CUtensorMap* tm_kv) {
   const int lane = threadIdx.x & 31;
   volatile int* abort = &s.abort_flag;
   uint64_t* full = is_v ? s.bar_vfull : s.bar_kfull;
   uint64_t* empty = is_v ? s.bar_vempty : s.bar_kempty;
+  uint64_t* land = kFp8 ? (is_v ? s.bar_vland : s.bar_kland) : full;
+  uint64_t* qland = kFp8 ? &s.bar_qland : &s.bar_qfull;
   Seg g;
   uint32_t it = 0, sidx = 0;
+  int pend_st = -1;  // 8-bit cache: a landed tile not yet converted (stage), its landing parity
+  uint32_t pend_ph = 0;
+  bool q_pend = false;
+  auto convert_pending = [&]() -> bool {
+    if (!kFp8 || pend_st < 0) return true;
+    if (!warp_wait(&land[pend_st], pend_ph, abort)) return false;
+    convert_stage_e4m3(is_v ? s.v[pend_st] : s.k[pend_st], lane);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&full[pend_st]);
+    pend_st = -1;
+    return true;
+  };
   const int nodes_per_tile = kBM / p.group;
   while (iter.next(s, p, g)) {
     const int npg = (g.P + g.N + kPage - 1) / kPage;
@@ -219,13 +291,14 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
     // the Q tiles go out while the page ids are on their way
     if (!is_v) {
       if (!warp_wait(&s.bar_qempty, (sidx & 1) ^ 1, abort)) return set_abort(s, p);
-      if (lane == 0) mbar_arrive_expect_tx(&s.bar_qfull, kAttnQTiles * kTileBytes);
+      if (lane == 0) mbar_arrive_expect_tx(qland, kAttnQTiles * kTileBytes);
       __syncwarp();
       if (lane < 2 * kAttnQTiles) {  // lane: Q tile lane / 2, half lane % 2
         const int qt = lane >> 1, half = lane & 1;
         const int node0 = g.off + (g.mp * kAttnQTiles + qt) * nodes_per_tile;
-        tma_load_3d(s.q[qt] + half * kHalfBytes, tm_q, &s.bar_qfull, half * 64, g.kvh * p.group, node0);
+        tma_load_3d(s.q[qt] + half * kHalfBytes, tm_q, qland, half * 64, g.kvh * p.group, node0);
       }
+      q_pend = kFp8;
     }
     for (int t = g.kb; t < g.ke; ++t, ++it) {
       const int st = it % kStages;
@@ -235,9 +308,9 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
         ids_cur = ids_next;
         ids_next = batch_ids(t + 4);
       }
-      // lane j < 16: page j / 2, 64-column half j % 2
-      int pid = __shfl_sync(0xffffffffu, ids_cur, bi * 8 + ((lane >> 1) & 7));
-      if (lane >= 2 * kPagesPerTile) pid = -1;
+      // bf16: lane j < 16 copies page j / 2, 64-column half j % 2; 8-bit: lane j < 8 copies page j (whole rows)
+      int pid = __shfl_sync(0xffffffffu, ids_cur, bi * 8 + (kFp8 ? (lane & 7) : ((lane >> 1) & 7)));
+      if (lane >= (kFp8 ? 1 : 2) * kPagesPerTile) pid = -1;
       const uint32_t mask = __ballot_sync(0xffffffffu, pid >= 0);
       const uint32_t bytes = static_cast<uint32_t>(__popc(mask)) * (kPage * 128u);
       if (!warp_wait(&empty[st], ph ^ 1, abort)) return set_abort(s, p);
@@ -249,27 +322,54 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
           if (*abort || globaltimer() - t0 > kWaitLimitNs) return set_abort(s, p);
         }
       }
-      if (lane == 0) mbar_arrive_expect_tx(&full[st], bytes);
+      if (lane == 0) mbar_arrive_expect_tx(&land[st], bytes);
       __syncwarp();
       if (pid >= 0) {
-        const int half = lane & 1;
-        uint8_t* dst = (is_v ? s.v[st] : s.k[st]) + half * kHalfBytes + (lane >> 1) * (kPage * 128);
-        tma_load_3d(dst, tm_kv, &full[st], half * 64, g.kvh, pid * kPage);
+        uint8_t* stage = is_v ? s.v[st] : s.k[st];
+        if (kFp8) {
+          tma_load_3d(stage + kHalfBytes + lane * (kPage * 128), tm_kv, &land[st], 0, g.kvh, pid * kPage);
+        } else {
+          const int half = lane & 1;
+          tma_load_3d(stage + half * kHalfBytes + (lane >> 1) * (kPage * 128), tm_kv, &land[st], half * 64, g.kvh,
+                      pid * kPage);
+        }
       }
       if (!is_v && it == 0) {
         __syncwarp();
         if (lane == 0) *reinterpret_cast<volatile int*>(&s.k_started) = 1;
       }
+      if (kFp8) {
+        // convert the previous tile while this one is on its way, then (segment start) the Q tiles
+        if (!convert_pending()) return set_abort(s, p);
+        pend_st = st;
+        pend_ph = ph;
+        if (q_pend) {
+          if (!warp_wait(&s.bar_qland, sidx & 1, abort)) return set_abort(s, p);
+          convert_q_bf16_f16(&s.q[0][0], kAttnQTiles * kTileBytes, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.bar_qfull);
+          q_pend = false;
+        }
+      }
     }
     ++sidx;
   }
+  if (!convert_pending()) return set_abort(s, p);
 }
 
 // ------------------------------------------------------------------------------------------------
 // Warp 1: tcgen05.mma issuer
 // ------------------------------------------------------------------------------------------------
+// Instruction descriptor of kind::f16 with f16 operands (the 8-bit cache path): the bf16 one with both operand
+// format fields (bits 7-9, 10-12) set to 0 = f16.
+__host__ __device__ constexpr uint32_t idesc_operands(uint32_t bf16_idesc, bool f16) {
+  return f16 ? (bf16_idesc & ~((7u << 7) | (7u << 10))) : bf16_idesc;
+}
+
+template <bool kFp8>
 __device__ __forceinline__ void issue_qk(const Smem& s, uint32_t tmem, int qt, int st) {
-  constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, false, false);
+  constexpr uint32_t idesc = idesc_operands(idesc_bf16_f32(kBM, kBN, false, false), kFp8);
   const uint32_t qaddr = smem_u32(s.q[qt]);
   const uint32_t kaddr = smem_u32(s.k[st]);
 #pragma unroll
@@ -280,8 +380,9 @@ __device__ __forceinline__ void issue_qk(const Smem& s, uint32_t tmem, int qt, i
   }
 }
 
+template <bool kFp8>
 __device__ __forceinline__ void issue_pv(const Smem& s, uint32_t tmem, int qt, int st, bool first) {
-  constexpr uint32_t idesc = idesc_bf16_f32(kBM, 128, false, true);
+  constexpr uint32_t idesc = idesc_operands(idesc_bf16_f32(kBM, 128, false, true), kFp8);
   const uint32_t vaddr = smem_u32(s.v[st]);
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk) {
@@ -290,6 +391,7 @@ __device__ __forceinline__ void issue_pv(const Smem& s, uint32_t tmem, int qt, i
   }
 }
 
+template <bool kFp8>
 __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t tmem) {
   const int lane = threadIdx.x & 31;
   volatile int* abort = &s.abort_flag;
@@ -303,9 +405,9 @@ __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t 
         if (!warp_wait(&s.bar_kfull[st], (it / kStages) & 1, abort)) return set_abort(s, p);
         tc_fence_after();
         if (lane == 0) {
-          issue_qk(s, tmem, 0, st);
+          issue_qk<kFp8>(s, tmem, 0, st);
           mma_commit(&s.bar_sfull[0]);
-          issue_qk(s, tmem, 1, st);
+          issue_qk<kFp8>(s, tmem, 1, st);
           mma_commit(&s.bar_sfull[1]);
           mma_commit(&s.bar_kempty[st]);
           if (t == g.ke - 1) mma_commit(&s.bar_qempty);
@@ -337,11 +439,11 @@ __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t 
         if (!warp_wait(&s.bar_pfull[qt], it & 1, abort)) return set_abort(s, p);
         tc_fence_after();
         if (lane == 0) {
-          issue_pv(s, tmem, qt, st, t == g.kb);
+          issue_pv<kFp8>(s, tmem, qt, st, t == g.kb);
           mma_commit(&s.bar_pvdone[qt]);
           if (qt == kAttnQTiles - 1) mma_commit(&s.bar_vempty[st]);
           if (has_next) {
-            issue_qk(s, tmem, qt, st1);
+            issue_qk<kFp8>(s, tmem, qt, st1);
             mma_commit(&s.bar_sfull[qt]);
             if (qt == kAttnQTiles - 1) {
               mma_commit(&s.bar_kempty[st1]);
@@ -509,6 +611,7 @@ __device__ bool build_ancestors(Smem& s, const AttnParams& p, const Seg& g) {
   return true;
 }
 
+template <bool kFp8>
 __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uint32_t tmem, int qt) {
   const int r = threadIdx.x - 128 - qt * kBM;  // row of M tile qt == TMEM lane
   const int wq = (threadIdx.x >> 5) & 3;
@@ -592,7 +695,12 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
           const float p0 = ex2_approx(y0), p1 = ex2_approx(y1);
           if ((c >> 1) & 1) acc1 = f2_add(acc1, f2_pack(p0, p1));
           else acc0 = f2_add(acc0, f2_pack(p0, p1));
-          pk[c >> 1] = pack_bf16x2_alu(p0, p1);
+          if (kFp8) {
+            const __half2 hp = __floats2half2_rn(p0, p1);  // the PV operands are f16 on this path
+            pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
+          } else {
+            pk[c >> 1] = pack_bf16x2_alu(p0, p1);
+          }
         }
         tmem_st16(lane_base + s_col + 16 * h, pk);
       }
@@ -628,7 +736,7 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
     const bool split = g.c0 != g.c1;
     const long long grow = static_cast<long long>(g.off + node) * p.hq + head;  // global row
     if (!split) {
-      const float inv_l = 1.f / l;
+      const float inv_l = p.v_scale / l;  // the V cache's scale (1 for a bf16 cache)
 #pragma unroll
       for (int cc = 0; cc < 128; cc += 32) {
         uint32_t o[32];
@@ -669,6 +777,7 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
   }
 }
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     tree_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -684,9 +793,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // tensor-map prefetches and the TMEM allocation.  The plan's barriers publish all of it.
   if (tid == 0) {
     mbar_init(&s.bar_qfull, 1);
+    mbar_init(&s.bar_qland, 1);
     mbar_init(&s.bar_qempty, 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&s.bar_kfull[i], 1);
+      mbar_init(&s.bar_kland[i], 1);
+      mbar_init(&s.bar_vland[i], 1);
       mbar_init(&s.bar_kempty[i], 1);
       mbar_init(&s.bar_vfull[i], 1);
       mbar_init(&s.bar_vempty[i], 1);
@@ -752,15 +864,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
     if (warp == 0 || warp == 2) {
-      kv_producer(s, p, iter, warp == 2, &tm_q, warp == 2 ? &tm_v : &tm_k);
+      kv_producer<kFp8>(s, p, iter, warp == 2, &tm_q, warp == 2 ? &tm_v : &tm_k);
     } else if (warp == 1) {
-      mma_issuer(s, p, iter, tmem);
+      mma_issuer<kFp8>(s, p, iter, tmem);
     } else {
       metadata(s, p, iter);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
-    softmax_epilogue(s, p, iter, tmem, warp < 8 ? 0 : 1);
+    softmax_epilogue<kFp8>(s, p, iter, tmem, warp < 8 ? 0 : 1);
   }
   tc_fence_before();
   __syncthreads();
@@ -883,7 +995,7 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
       M = Mb;
     }
     if (!ok) continue;
-    const float inv = 1.f / L;
+    const float inv = p.v_scale / L;  // the V cache's scale (1 for a bf16 cache)
     uint2* dst = reinterpret_cast<uint2*>(p.out + grow * 128 + q0 * 4);
 #pragma unroll
     for (int q = 0; q < kCombineQuads; ++q)
@@ -898,19 +1010,24 @@ static_assert(sizeof(attn::Smem) + 1024 <= 227 * 1024, "shared memory of one CTA
 size_t attention_smem_bytes() { return sizeof(attn::Smem) + 1024; }
 
 cudaError_t launch_tree_attention(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                                  const AttnParams& p, int grid, cudaStream_t stream) {
+                                  const AttnParams& p, int grid, bool fp8_cache, cudaStream_t stream) {
   static std::atomic<bool> attr_set[kMaxDevices];
   const int dev = current_device();
   if (dev < 0) return cudaErrorInvalidDevice;
   const size_t smem = attention_smem_bytes();
   if (!attr_set[dev].load(std::memory_order_acquire)) {
-    cudaError_t e = cudaFuncSetAttribute(attn::tree_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = cudaFuncSetAttribute(attn::tree_attention_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn::tree_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  cudaError_t e = launch_pdl(attn::tree_attention_kernel, dim3(grid), dim3(attn::kThreads), smem, stream, nullptr,
-                             tm_q, tm_k, tm_v, p);
+  cudaError_t e = fp8_cache ? launch_pdl(attn::tree_attention_kernel<true>, dim3(grid), dim3(attn::kThreads), smem,
+                                         stream, nullptr, tm_q, tm_k, tm_v, p)
+                            : launch_pdl(attn::tree_attention_kernel<false>, dim3(grid), dim3(attn::kThreads), smem,
+                                         stream, nullptr, tm_q, tm_k, tm_v, p);
   if (e != cudaSuccess) return e;
   // The combine kernel may start as soon as the attention grid is scheduled; its griddepcontrol.wait
   // holds it until the attention grid has finished and its writes are visible.

@@ -150,6 +150,13 @@ def attention_inputs(seed: int, num_q_heads: int, num_kv_heads: int, prefix_lens
                            num_q_heads=num_q_heads, num_kv_heads=num_kv_heads)
 
 
+def e4m3_cache(values: np.ndarray, scale: float) -> np.ndarray:
+    """8-bit E4M3 codes (uint8) of a synthetic cache: values / scale converted by torch's float8_e4m3fn cast
+    (round to nearest even).  Values must stay within +-448 * scale."""
+    x = torch.from_numpy(np.ascontiguousarray(values, dtype=np.float32) / np.float32(scale))
+    return x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
 def plant_tree_values(inp: AttentionInputs, magnitude: float = 8.0, base_scale: float = 0.5,
                       seed: int = 0) -> AttentionInputs:
     """Planted-V probe: every tree slot j of every sequence gets V = magnitude * e_(j mod D) in each
