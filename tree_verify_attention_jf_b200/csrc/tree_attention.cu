@@ -288,6 +288,9 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
     };
     int ids_cur = batch_ids(g.kb);
     int ids_next = batch_ids(g.kb + 4);
+    // 8-bit cache: the previous segment's last tile is converted now -- the Q buffer frees only after that
+    // tile's QK has run
+    if (!convert_pending()) return set_abort(s, p);
     // the Q tiles go out while the page ids are on their way
     if (!is_v) {
       if (!warp_wait(&s.bar_qempty, (sidx & 1) ^ 1, abort)) return set_abort(s, p);
