@@ -198,35 +198,42 @@ __device__ void build_plan(Smem& s, const AttnParams& p) {
 // ------------------------------------------------------------------------------------------------
 // One K or V stage: the copy put the tile's 8-bit rows (128 keys x 128 dims, one 128-byte row per key) in the
 // stage's upper 16 KB; they become f16 in the 128-byte-swizzled [half][128 keys][64 dims] layout of the whole
-// stage.  A warp converts four rows per step: all lanes read their 16 bytes first, then write 2 x 16 bytes;
-// the writes of a step land in rows [0, 16 KB) and on the 8-bit rows the same step has just read, so rows
-// still to be read are never overwritten.
+// stage.  A warp converts 16 rows per step (4 chunks of 16 bytes per lane, all read before any is written): the
+// writes of a step land in rows [0, 16 KB) and on the 8-bit rows the same step has just read, so rows still to
+// be read are never overwritten.
 __device__ __forceinline__ void convert_stage_e4m3(uint8_t* stage, int lane) {
   const int c = lane & 7;  // 16-byte chunk of the 8-bit row: dims [16 c, 16 c + 16)
-  for (int r0 = 0; r0 < kBN; r0 += 4) {
-    const int row = r0 + (lane >> 3);
-    const uint4 raw = *reinterpret_cast<const uint4*>(stage + kHalfBytes + row * 128 + c * 16);
-    __syncwarp();
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint32_t hv[8];
+  const int j0 = 2 * (c & 3);  // its f16 bytes are chunks j0, j0 + 1 of half c / 4
+  for (int r0 = 0; r0 < kBN; r0 += 16) {
+    uint4 raw[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xffffu), __NV_E4M3);
-      const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
-      hv[2 * i] = static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16);
-      hv[2 * i + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
+    for (int k = 0; k < 4; ++k)
+      raw[k] = *reinterpret_cast<const uint4*>(stage + kHalfBytes + (r0 + (lane >> 3) + 4 * k) * 128 + c * 16);
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int row = r0 + (lane >> 3) + 4 * k;
+      const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+      uint32_t hv[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __half2_raw lo =
+            __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xffffu), __NV_E4M3);
+        const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
+        hv[2 * i] = static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16);
+        hv[2 * i + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
+      }
+      uint8_t* base = stage + (c >> 2) * kHalfBytes + row * 128;
+      *reinterpret_cast<uint4*>(base + ((j0 ^ (row & 7)) * 16)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      *reinterpret_cast<uint4*>(base + (((j0 + 1) ^ (row & 7)) * 16)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
     }
-    // dims [16 c, 16 c + 16) are f16 bytes [32 (c % 4), 32 (c % 4) + 32) of half c / 4: chunks 2 (c % 4) and + 1
-    const int j0 = 2 * (c & 3);
-    uint8_t* base = stage + (c >> 2) * kHalfBytes + row * 128;
-    *reinterpret_cast<uint4*>(base + ((j0 ^ (row & 7)) * 16)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    *reinterpret_cast<uint4*>(base + (((j0 + 1) ^ (row & 7)) * 16)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
     __syncwarp();
   }
 }
 
 // The Q tiles in place, bf16 -> f16, element by element (the swizzle does not matter).
 __device__ __forceinline__ void convert_q_bf16_f16(uint8_t* q, int bytes, int lane) {
+#pragma unroll 4
   for (int i = lane * 16; i < bytes; i += 32 * 16) {
     uint4 v = *reinterpret_cast<const uint4*>(q + i);
     uint32_t w[4] = {v.x, v.y, v.z, v.w};

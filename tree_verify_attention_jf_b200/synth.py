@@ -153,8 +153,10 @@ def attention_inputs(seed: int, num_q_heads: int, num_kv_heads: int, prefix_lens
 def e4m3_cache(values: np.ndarray, scale: float) -> np.ndarray:
     """8-bit E4M3 codes (uint8) of a synthetic cache: values / scale converted by torch's float8_e4m3fn cast
     (round to nearest even).  Values must stay within +-448 * scale."""
-    x = torch.from_numpy(np.ascontiguousarray(values, dtype=np.float32) / np.float32(scale))
-    return x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    x = np.ascontiguousarray(values, dtype=np.float32) / np.float32(scale)
+    if np.abs(x).max(initial=0.0) > 448.0:
+        raise ValueError("values / scale exceed the E4M3 range (448)")
+    return torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
 def plant_tree_values(inp: AttentionInputs, magnitude: float = 8.0, base_scale: float = 0.5,
