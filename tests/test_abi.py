@@ -23,6 +23,14 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, n), n
 
 
+def test_debug_build_exports_every_declared_symbol():
+    D = _lib.debug_lib()
+    for n in _lib.declared_functions() + _lib.declared_functions(_lib.DEBUG_HEADER):
+        assert hasattr(D, n), n
+    assert _lib.declared_functions(_lib.DEBUG_HEADER) == ["jf_debug_hold"]
+    assert not hasattr(_lib.lib(), "jf_debug_hold")  # the release build has no test hooks
+
+
 def test_status_strings(L):
     assert _lib.status_string(0) == "JF_OK"
     assert _lib.status_string(4) == "JF_ERR_DEVICE_CHECK"

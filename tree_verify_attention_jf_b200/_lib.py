@@ -9,7 +9,9 @@ import re
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libjf.so")
+DEBUG_LIB_PATH = os.path.join(_PKG, "libjf_debug.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "jf.h")
+DEBUG_HEADER = os.path.join(os.path.dirname(_PKG), "include", "jf_debug.h")
 
 JF_OK = 0
 JF_ERR_INVALID_ARG = 1
@@ -33,9 +35,27 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m tree_verify_attention_jf_b200.build`")
-    L = ctypes.CDLL(LIB_PATH)
+    _lib = _load(LIB_PATH)
+    return _lib
+
+
+_debug_lib = None
+
+
+def debug_lib() -> ctypes.CDLL:
+    """The debug build libjf_debug.so (50 ms wait limit, jf_debug.h hooks), for the failure-detection tests."""
+    global _debug_lib
+    if _debug_lib is None:
+        _debug_lib = _load(DEBUG_LIB_PATH)
+        _debug_lib.jf_debug_hold.argtypes = [ctypes.c_int]
+        _debug_lib.jf_debug_hold.restype = ctypes.c_int
+    return _debug_lib
+
+
+def _load(path: str) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m tree_verify_attention_jf_b200.build`")
+    L = ctypes.CDLL(path)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.jf_status_string.argtypes = [i]
     L.jf_status_string.restype = ctypes.c_char_p
@@ -64,7 +84,6 @@ def lib() -> ctypes.CDLL:
     L.jf_commit_kv.restype = i
     L.jf_tree_kv_append.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, f, vp, vp]
     L.jf_tree_kv_append.restype = i
-    _lib = L
     return L
 
 
@@ -72,9 +91,9 @@ def status_string(code: int) -> str:
     return lib().jf_status_string(int(code)).decode()
 
 
-def declared_functions() -> list[str]:
-    """Names of the functions include/jf.h declares (used to check the library's exports)."""
-    text = open(HEADER).read()
+def declared_functions(header: str = HEADER) -> list[str]:
+    """Names of the functions a header declares (used to check the library's exports)."""
+    text = open(header).read()
     return sorted(set(re.findall(r"JF_API\s+[\w\s\*]+?\b(jf_\w+)\s*\(", text)))
 
 

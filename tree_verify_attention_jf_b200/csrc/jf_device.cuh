@@ -13,8 +13,13 @@
 namespace jf {
 
 // A bounded device wait gives up after this many nanoseconds of %globaltimer and reports
-// JF_ERR_TIMEOUT.  Far above any legitimate wait in these kernels (microseconds).
+// JF_ERR_TIMEOUT.  Far above any legitimate wait in these kernels (microseconds).  The debug build
+// (JF_DEBUG) uses 50 ms, so that a test can make a wait run out quickly.
+#ifdef JF_DEBUG
+constexpr uint64_t kWaitLimitNs = 50000000ull;
+#else
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+#endif
 
 __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);

@@ -34,6 +34,12 @@
 #include "jf_internal.h"
 
 namespace jf {
+#ifdef JF_DEBUG
+// Debug build only: while g_debug_hold is nonzero, every attention CTA first waits for it to clear.  Nothing
+// clears it during a call, so the wait runs out -- before any copy or MMA is issued -- and the call must come
+// back with JF_ERR_TIMEOUT in dev_status and the context still usable (set by jf_debug_hold).
+__device__ int g_debug_hold;
+#endif
 namespace attn {
 
 constexpr int kPage = 16;
@@ -66,6 +72,7 @@ struct __align__(1024) Smem {
   uint64_t bar_qland, bar_kland[kStages], bar_vland[kStages];
   uint64_t bar_sfull[kAttnQTiles], bar_pfull[kAttnQTiles], bar_pvdone[kAttnQTiles];
   uint64_t bar_metafull[2], bar_metaempty[2];
+  uint64_t bar_drain;  // the MMA warp's last MMA, waited for when unwinding after an abort
   uint32_t tmem_base;
   int meta_valid[2];
   int meta_ctl;
@@ -136,6 +143,15 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ void set_abort(Smem& s, const AttnParams& p) {
   *reinterpret_cast<volatile int*>(&s.abort_flag) = 1;
   report(p.status, JF_ERR_TIMEOUT);
+}
+
+// While unwinding after an abort: waits up to `ns` for a phase, ignoring the abort flag, so that copies and
+// MMAs already issued finish before the CTA releases its tensor memory and exits.
+constexpr uint64_t kDrainNs = kWaitLimitNs;
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > kDrainNs) return;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -265,6 +281,15 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
   int pend_st = -1;  // 8-bit cache: a landed tile not yet converted (stage), its landing parity
   uint32_t pend_ph = 0;
   bool q_pend = false;
+  // the latest phase this warp armed on each landing barrier (bit st of armed; its parity in armed_par), and on
+  // the Q landing barrier: on an abort the warp waits for them, i.e. for every copy it issued
+  uint32_t armed = 0, armed_par = 0, q_armed = 0, q_par = 0;
+  auto unwind = [&]() {
+    set_abort(s, p);
+    for (int st = 0; st < kStages; ++st)
+      if (armed & (1u << st)) drain_wait(&land[st], (armed_par >> st) & 1u);
+    if (q_armed) drain_wait(qland, q_par);
+  };
   auto convert_pending = [&]() -> bool {
     if (!kFp8 || pend_st < 0) return true;
     if (!warp_wait(&land[pend_st], pend_ph, abort)) return false;
@@ -297,11 +322,13 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
     int ids_next = batch_ids(g.kb + 4);
     // 8-bit cache: the previous segment's last tile is converted now -- the Q buffer frees only after that
     // tile's QK has run
-    if (!convert_pending()) return set_abort(s, p);
+    if (!convert_pending()) return unwind();
     // the Q tiles go out while the page ids are on their way
     if (!is_v) {
-      if (!warp_wait(&s.bar_qempty, (sidx & 1) ^ 1, abort)) return set_abort(s, p);
+      if (!warp_wait(&s.bar_qempty, (sidx & 1) ^ 1, abort)) return unwind();
       if (lane == 0) mbar_arrive_expect_tx(qland, kAttnQTiles * kTileBytes);
+      q_armed = 1;
+      q_par = sidx & 1;
       __syncwarp();
       if (lane < 2 * kAttnQTiles) {  // lane: Q tile lane / 2, half lane % 2
         const int qt = lane >> 1, half = lane & 1;
@@ -323,16 +350,18 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
       if (lane >= (kFp8 ? 1 : 2) * kPagesPerTile) pid = -1;
       const uint32_t mask = __ballot_sync(0xffffffffu, pid >= 0);
       const uint32_t bytes = static_cast<uint32_t>(__popc(mask)) * (kPage * 128u);
-      if (!warp_wait(&empty[st], ph ^ 1, abort)) return set_abort(s, p);
+      if (!warp_wait(&empty[st], ph ^ 1, abort)) return unwind();
       if (is_v && it == 0) {
         // The copy engine serves requests in order and the first S needs Q and K only: the kernel's
         // first V tile is queued behind the first K tile (bounded wait, like every other).
         const uint64_t t0 = globaltimer();
         while (*reinterpret_cast<volatile int*>(&s.k_started) == 0) {
-          if (*abort || globaltimer() - t0 > kWaitLimitNs) return set_abort(s, p);
+          if (*abort || globaltimer() - t0 > kWaitLimitNs) return unwind();
         }
       }
       if (lane == 0) mbar_arrive_expect_tx(&land[st], bytes);
+      armed |= 1u << st;
+      armed_par = (armed_par & ~(1u << st)) | (ph << st);
       __syncwarp();
       if (pid >= 0) {
         uint8_t* stage = is_v ? s.v[st] : s.k[st];
@@ -350,11 +379,11 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
       }
       if (kFp8) {
         // convert the previous tile while this one is on its way, then (segment start) the Q tiles
-        if (!convert_pending()) return set_abort(s, p);
+        if (!convert_pending()) return unwind();
         pend_st = st;
         pend_ph = ph;
         if (q_pend) {
-          if (!warp_wait(&s.bar_qland, sidx & 1, abort)) return set_abort(s, p);
+          if (!warp_wait(&s.bar_qland, sidx & 1, abort)) return unwind();
           convert_q_bf16_f16(&s.q[0][0], kAttnQTiles * kTileBytes, lane);
           fence_proxy_async_smem();
           __syncwarp();
@@ -365,7 +394,7 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
     }
     ++sidx;
   }
-  if (!convert_pending()) return set_abort(s, p);
+  if (!convert_pending()) return unwind();
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -407,12 +436,21 @@ __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t 
   volatile int* abort = &s.abort_flag;
   Seg g;
   uint32_t it = 0, sidx = 0;
+  bool issued = false;
+  auto unwind = [&]() {  // the last MMA issued completes before the CTA releases its tensor memory
+    set_abort(s, p);
+    if (issued) {
+      if (lane == 0) mma_commit(&s.bar_drain);
+      __syncwarp();
+      drain_wait(&s.bar_drain, 0);
+    }
+  };
   while (iter.next(s, p, g)) {
-    if (!warp_wait(&s.bar_qfull, sidx & 1, abort)) return set_abort(s, p);
+    if (!warp_wait(&s.bar_qfull, sidx & 1, abort)) return unwind();
     for (int t = g.kb; t < g.ke; ++t, ++it) {
       const int st = it % kStages;
       if (t == g.kb) {  // S of the segment's first tile for both Q tiles
-        if (!warp_wait(&s.bar_kfull[st], (it / kStages) & 1, abort)) return set_abort(s, p);
+        if (!warp_wait(&s.bar_kfull[st], (it / kStages) & 1, abort)) return unwind();
         tc_fence_after();
         if (lane == 0) {
           issue_qk<kFp8>(s, tmem, 0, st);
@@ -423,11 +461,12 @@ __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t 
           if (t == g.ke - 1) mma_commit(&s.bar_qempty);
         }
         __syncwarp();
+        issued = true;
       }
       const bool has_next = t + 1 < g.ke;
       const int st1 = (it + 1) % kStages;
-      if (has_next && !warp_wait(&s.bar_kfull[st1], ((it + 1) / kStages) & 1, abort)) return set_abort(s, p);
-      if (!warp_wait(&s.bar_vfull[st], (it / kStages) & 1, abort)) return set_abort(s, p);
+      if (has_next && !warp_wait(&s.bar_kfull[st1], ((it + 1) / kStages) & 1, abort)) return unwind();
+      if (!warp_wait(&s.bar_vfull[st], (it / kStages) & 1, abort)) return unwind();
       const int zf = g.P + g.N - t * kBN;  // first row of this tile past the sequence
       if (zf < kBN) {
         // Keys beyond the sequence's last slot: clear their V rows so stale cache contents (even NaN)
@@ -446,7 +485,7 @@ __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t 
         __syncwarp();
       }
       for (int qt = 0; qt < kAttnQTiles; ++qt) {
-        if (!warp_wait(&s.bar_pfull[qt], it & 1, abort)) return set_abort(s, p);
+        if (!warp_wait(&s.bar_pfull[qt], it & 1, abort)) return unwind();
         tc_fence_after();
         if (lane == 0) {
           issue_pv<kFp8>(s, tmem, qt, st, t == g.kb);
@@ -462,6 +501,7 @@ __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t 
           }
         }
         __syncwarp();
+        issued = true;
       }
     }
     ++sidx;
@@ -621,6 +661,8 @@ __device__ bool build_ancestors(Smem& s, const AttnParams& p, const Seg& g) {
   return true;
 }
 
+// A warp whose wait gives up (ok = false) keeps walking the segments with its work skipped, so that the
+// ancestor build's named barriers are still reached by all 256 softmax threads; it reports the abort once.
 template <bool kFp8>
 __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uint32_t tmem, int qt) {
   const int r = threadIdx.x - 128 - qt * kBM;  // row of M tile qt == TMEM lane
@@ -633,17 +675,22 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
   const int nodes_per_tile = kBM / p.group;
   Seg g;
   uint32_t it = 0, sidx = 0;
+  bool ok = true;
   while (iter.next(s, p, g)) {
     const int buf = sidx & 1;
     const int node = (g.mp * kAttnQTiles + qt) * nodes_per_tile + r / p.group;
     const int head = g.kvh * p.group + (r % p.group);
     const bool row_valid = node < g.N;
-    if (static_cast<long long>(g.ke) * kBN > g.P && !build_ancestors(s, p, g)) return set_abort(s, p);
+    if (static_cast<long long>(g.ke) * kBN > g.P && !build_ancestors(s, p, g)) ok = false;
     const uint32_t* anc = &s.anc[row_valid ? node : 0][0];
     float m_use = -INFINITY, l = 0.f;
     for (int t = g.kb; t < g.ke; ++t, ++it) {
       const bool tree_tile = (t + 1) * kBN > g.P;
-      if (!warp_wait(&s.bar_sfull[qt], it & 1, abort)) return set_abort(s, p);
+      if (!ok) continue;
+      if (!warp_wait(&s.bar_sfull[qt], it & 1, abort)) {
+        ok = false;
+        continue;
+      }
       // S_qt(it) ready also means PV_qt(it-1) is complete: its commit tracks every earlier MMA.
       tc_fence_after();
       // The row of S in registers, in two halves: the max of the first half is taken while the
@@ -738,9 +785,13 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
       mbar_arrive(&s.bar_pfull[qt]);
     }
     // ---------------- epilogue of the segment
-    if (!warp_wait(&s.bar_metafull[buf], (sidx >> 1) & 1, abort)) return set_abort(s, p);
+    if (ok && !warp_wait(&s.bar_metafull[buf], (sidx >> 1) & 1, abort)) ok = false;
     const bool seg_ok = s.meta_valid[buf] != 0;
-    if (!warp_wait(&s.bar_pvdone[qt], (it - 1) & 1, abort)) return set_abort(s, p);
+    if (ok && !warp_wait(&s.bar_pvdone[qt], (it - 1) & 1, abort)) ok = false;
+    if (!ok) {
+      ++sidx;
+      continue;
+    }
     tc_fence_after();
     mbar_arrive(&s.bar_metaempty[buf]);
     const bool split = g.c0 != g.c1;
@@ -785,6 +836,7 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
     }
     ++sidx;
   }
+  if (!ok) set_abort(s, p);
 }
 
 template <bool kFp8>
@@ -818,6 +870,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.bar_pfull[i], kBM);
       mbar_init(&s.bar_pvdone[i], 1);
     }
+    mbar_init(&s.bar_drain, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.bar_metafull[i], 32);
       mbar_init(&s.bar_metaempty[i], kAttnQTiles * kBM);
@@ -841,10 +894,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Slot blockIdx.x of the split-unit table is written only by this CTA (if it starts a split unit);
   // clear what an earlier call left there.
   if (tid == 0 && blockIdx.x < kMaxGrid) p.units[blockIdx.x] = make_int4(0, 0, 0, 0);
+#ifdef JF_DEBUG
+  if (tid == 0 && *reinterpret_cast<volatile int*>(&g_debug_hold) != 0) {
+    const uint64_t t0 = globaltimer();
+    while (*reinterpret_cast<volatile int*>(&g_debug_hold) != 0) {
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        set_abort(s, p);
+        break;
+      }
+    }
+  }
+#endif
   build_plan(s, p);
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  bool idle = s.bad_meta != 0;
+  bool idle = s.bad_meta != 0 || s.abort_flag != 0;  // abort_flag: set above by the debug build only
   if (idle && blockIdx.x == 0 && tid == 0) report(p.status, JF_ERR_DEVICE_CHECK);
   const long long W = s.cum_work[p.batch];
   const int G = static_cast<int>(W < static_cast<long long>(gridDim.x) ? W : static_cast<long long>(gridDim.x));
@@ -1045,3 +1109,10 @@ cudaError_t launch_tree_attention(const CUtensorMap& tm_q, const CUtensorMap& tm
 }
 
 }  // namespace jf
+
+#ifdef JF_DEBUG
+extern "C" JF_API jf_status jf_debug_hold(int on) {
+  const int v = on ? 1 : 0;
+  return cudaMemcpyToSymbol(jf::g_debug_hold, &v, sizeof(v)) == cudaSuccess ? JF_OK : JF_ERR_CUDA;
+}
+#endif
