@@ -3,14 +3,22 @@ device plan): every (unit, kv tile) pair is covered exactly once, a unit's shari
 those that hold one of its kv tiles, partial slots never collide, every CTA's range is non-empty, and
 a CTA that starts segments in mid-range gets correspondingly fewer kv tiles.
 
-Each unit costs SEG_COST + kt positions: SEG_COST leading positions (the price of starting a segment
-in mid-kernel) and then its kt kv tiles."""
+A unit is one (sequence, kv head, pair of 128-row M tiles).  It costs SEG_COST + kt positions: SEG_COST
+leading positions (the price of starting a segment in mid-kernel) and then its kt positions, position t
+reading kv tile (t - rot) mod kt, rot being where the owner of the unit's last position starts."""
+
+import collections
 
 import numpy as np
 import pytest
 
 BN, BM = 128, 128
 SEG_COST = 3
+Q_TILES = 2  # M tiles per unit
+
+
+def pairs(N, group):
+    return ((N * group + BM - 1) // BM + Q_TILES - 1) // Q_TILES
 
 
 def plan(prefix, nodes, hkv, group):
@@ -20,8 +28,7 @@ def plan(prefix, nodes, hkv, group):
             work.append(0)
             continue
         kt = (P + N + BN - 1) // BN
-        mt = (N * group + BM - 1) // BM
-        work.append(hkv * mt * (kt + SEG_COST))
+        work.append(hkv * pairs(N, group) * (kt + SEG_COST))
     cum = np.concatenate([[0], np.cumsum(work)]).astype(np.int64)
     return cum
 
@@ -41,7 +48,7 @@ def segments(prefix, nodes, hkv, group, grid):
                 b += 1
             P, N = prefix[b], nodes[b]
             kt = (P + N + BN - 1) // BN
-            mtn = (N * group + BM - 1) // BM
+            mtn = pairs(N, group)
             span = kt + SEG_COST
             unit = (x - cum[b]) // span
             u0, u1 = cum[b] + unit * span, cum[b] + unit * span + span
@@ -52,8 +59,10 @@ def segments(prefix, nodes, hkv, group, grid):
                 continue
             c0, c1 = cta_of(u0 + SEG_COST), cta_of(u1 - 1)
             slot = 2 * c + 1 if c == c0 else 2 * c
+            rot = max(c1 * W // G - u0 - SEG_COST, 0)
             out.append(dict(cta=c, b=b, kvh=unit // mtn, mt=unit % mtn, kb=max(t0, 0), ke=t1, c0=c0, c1=c1,
-                            slot=slot, range=(c * W // G, (c + 1) * W // G)))
+                            slot=slot, range=(c * W // G, (c + 1) * W // G), kt=kt, rot=rot,
+                            start=u0 + SEG_COST - c * W // G))  # local time of position 0
     return out, W, G
 
 
@@ -69,14 +78,18 @@ def test_cover_exactly_once(prefix, nodes, hkv, group, grid):
     segs, W, G = segments(prefix, nodes, hkv, group, grid)
     seen = {}
     for s in segs:
+        assert 0 <= s["rot"] < s["kt"]
         for t in range(s["kb"], s["ke"]):
-            key = (s["b"], s["kvh"], s["mt"], t)
+            key = (s["b"], s["kvh"], s["mt"], (t - s["rot"]) % s["kt"])
             assert key not in seen
             seen[key] = s["cta"]
-    tiles = sum(hkv * ((N * group + BM - 1) // BM) * ((P + N + BN - 1) // BN)
-                for P, N in zip(prefix, nodes) if N > 0)
+    tiles = sum(hkv * pairs(N, group) * ((P + N + BN - 1) // BN) for P, N in zip(prefix, nodes) if N > 0)
     assert len(seen) == tiles
-    assert W == tiles + SEG_COST * sum(hkv * ((N * group + BM - 1) // BM) for N in nodes if N > 0)
+    assert W == tiles + SEG_COST * sum(hkv * pairs(N, group) for N in nodes if N > 0)
+    # the pieces of a unit agree on its rotation, and the owner of the last position reads tile 0 first
+    for s in segs:
+        if s["cta"] == s["c1"] and s["c0"] != s["c1"]:
+            assert (s["kb"] - s["rot"]) % s["kt"] == 0
     per_cta = {}
     for s in segs:
         per_cta.setdefault(s["cta"], []).append(s)
@@ -96,3 +109,24 @@ def test_cover_exactly_once(prefix, nodes, hkv, group, grid):
                 assert x["slot"] not in slots
                 slots.add(x["slot"])
                 assert x["slot"] < 2 * G
+
+
+def test_pairs_of_one_kv_head_read_in_step():
+    """Qwen3-30B-A3B shape (4 sequences, 32768-token prefix, 256-node trees, 4 kv heads, 8 q heads per kv
+    head: 8 units per (sequence, kv head)): at every CTA-local time the units of one (sequence, kv head)
+    read tile x or tile x + (kt - W / G) (rounding: +-1), x the local time, with a few reads two such
+    steps ahead (a CTA whose range lies inside one unit)."""
+    segs, W, G = segments([32768] * 4, [256] * 4, 4, 8, 148)
+    kt = segs[0]["kt"]
+    lag = kt - W // G
+    phases = collections.defaultdict(collections.Counter)
+    for s in segs:
+        for t in range(s["kb"], s["ke"]):
+            tau = s["start"] + t  # CTA-local time of this position
+            phases[(s["b"], s["kvh"])][((t - s["rot"]) % kt - tau) % kt] += 1
+    assert len(phases) == 16
+    for grp, c in phases.items():
+        assert sum(c.values()) == 8 * kt
+        main = sum(v for k, v in c.items() if k in (0, lag - 1, lag, lag + 1))
+        assert main >= 0.95 * 8 * kt, (grp, sorted(c.items()))
+        assert set(c) <= {0, lag - 1, lag, lag + 1, 2 * lag - 2, 2 * lag - 1, 2 * lag, 2 * lag + 1}, sorted(c.items())

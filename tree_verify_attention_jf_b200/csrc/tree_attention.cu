@@ -82,9 +82,14 @@ struct __align__(1024) Smem {
 };
 
 struct Seg {
-  int b, kvh, mp, kb, ke;  // kv tiles [kb, ke) of unit (b, kvh, M-tile pair mp)
+  int b, kvh, mp, kb, ke;  // positions [kb, ke) of unit (b, kvh, M-tile pair mp)
   int P, N, off, kt;       // prefix length, nodes, first global node, kv tiles of the sequence
   int c0, c1, slot;        // CTAs sharing the unit; this CTA's partial slot (times kAttnQTiles)
+  int rot;                 // the unit's rotation: position t reads kv tile (t - rot) mod kt
+  __device__ __forceinline__ int tile(int t) const {
+    const int x = t - rot;
+    return x < 0 ? x + kt : x;
+  }
 };
 
 __device__ __forceinline__ int cta_of(long long x, long long W, int G) {
@@ -96,11 +101,17 @@ __device__ __forceinline__ int pairs_of(int N, int group) {
   return (mtn + kAttnQTiles - 1) / kAttnQTiles;
 }
 
-// Cost space: a unit costs kSegCost + kt, its kv tiles preceded by kSegCost positions that stand for
-// the time a CTA loses when it starts a segment in mid-kernel (the previous segment's epilogue, the Q
-// reload, the refill of the K/V pipeline).  Cutting this space into equal ranges gives a CTA that
-// crosses a unit boundary correspondingly fewer kv tiles.  A CTA whose range ends inside a unit's
-// leading positions takes no part in that unit.
+// Cost space: a unit costs kSegCost + kt, its kt positions preceded by kSegCost that stand for the time a
+// CTA loses when it starts a segment in mid-kernel (the previous segment's epilogue, the Q reload, the refill
+// of the K/V pipeline).  Cutting this space into equal ranges gives a CTA that crosses a unit boundary
+// correspondingly fewer kv tiles.  A CTA whose range ends inside a unit's leading positions takes no part in
+// that unit.
+//
+// Positions map to kv tiles through a rotation per unit, chosen so that the CTA owning the unit's last
+// position starts its range on kv tile 0.  Every CTA starts at the same time and moves at about the same
+// rate, so at local time x a CTA reads tile x or tile x + (kt - W / G) of its unit: the M-tile pairs of one
+// (sequence, kv head), which read the same K and V, do so at two offsets instead of one offset each, and the
+// later readers find most of the tiles in L2.  Any rotation keeps the pieces of a unit disjoint.
 struct SegIter {
   long long x, xend, W;
   int G, b;
@@ -127,6 +138,8 @@ struct SegIter {
       g.c0 = cta_of(u0 + kSegCost, W, G);  // owner of the unit's first kv tile
       g.c1 = cta_of(u1 - 1, W, G);         // owner of its last
       g.slot = (static_cast<int>(blockIdx.x) == g.c0) ? 2 * blockIdx.x + 1 : 2 * blockIdx.x;
+      const long long k1 = static_cast<long long>(g.c1) * W / G - u0 - kSegCost;  // where the owner of the last starts
+      g.rot = k1 > 0 ? static_cast<int>(k1) : 0;
       return true;
     }
     return false;
@@ -304,13 +317,13 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
   while (iter.next(s, p, g)) {
     const int npg = (g.P + g.N + kPage - 1) / kPage;
     const int32_t* bt = p.block_table + static_cast<long long>(g.b) * p.max_pages;
-    // Page ids are fetched four tiles at a time (lane l: logical page 8 * (t0 + l / 8) + l % 8, -1 = not
+    // Page ids are fetched four positions at a time (lane l: logical page 8 * tile(t0 + l / 8) + l % 8, -1 = not
     // loaded) and one batch ahead, so the block-table latency stays off the issue path.
     auto batch_ids = [&](int t0) {
       int pid = -1;
       const int t = t0 + (lane >> 3);
       if (t < g.ke) {
-        const int pg = t * kPagesPerTile + (lane & 7);
+        const int pg = g.tile(t) * kPagesPerTile + (lane & 7);
         if (pg < npg && pg < p.max_pages) {
           const int v = __ldg(bt + pg);
           if (v >= 0 && v < p.num_pages) pid = v;
@@ -467,7 +480,7 @@ __device__ void mma_issuer(Smem& s, const AttnParams& p, SegIter iter, uint32_t 
       const int st1 = (it + 1) % kStages;
       if (has_next && !warp_wait(&s.bar_kfull[st1], ((it + 1) / kStages) & 1, abort)) return unwind();
       if (!warp_wait(&s.bar_vfull[st], (it / kStages) & 1, abort)) return unwind();
-      const int zf = g.P + g.N - t * kBN;  // first row of this tile past the sequence
+      const int zf = g.P + g.N - g.tile(t) * kBN;  // first row of this tile past the sequence
       if (zf < kBN) {
         // Keys beyond the sequence's last slot: clear their V rows so stale cache contents (even NaN)
         // cannot reach the output through 0 * V.  A whole 128-byte row is cleared, so the swizzle does
@@ -536,17 +549,23 @@ __device__ void metadata(Smem& s, const AttnParams& p, SegIter iter) {
       const int i = lane + 32 * k;
       pr[k] = i < g.N ? __ldg(par + i) : -1;
     }
-    int pg1 = g.ke * kPagesPerTile;
-    if (pg1 > npg) pg1 = npg;
-    if (pg1 > p.max_pages) pg1 = p.max_pages;
     int bad = (static_cast<long long>(g.P) + g.N > static_cast<long long>(p.max_pages) * kPage) ? 1 : 0;
-    for (int pg = g.kb * kPagesPerTile + lane; pg < pg1; pg += 4 * 32) {
-      int v[4];
+    // the segment's tiles: [a, a + len) of the unit, wrapped at kt
+    const int a = g.tile(g.kb), len = g.ke - g.kb;
+    const int first_end = a + len < g.kt ? a + len : g.kt;
+    for (int part = 0; part < 2; ++part) {
+      const int t0 = part == 0 ? a : 0, t1 = part == 0 ? first_end : a + len - g.kt;
+      int pg1 = t1 * kPagesPerTile;
+      if (pg1 > npg) pg1 = npg;
+      if (pg1 > p.max_pages) pg1 = p.max_pages;
+      for (int pg = t0 * kPagesPerTile + lane; pg < pg1; pg += 4 * 32) {
+        int v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = (pg + 32 * u < pg1) ? __ldg(bt + pg + 32 * u) : 0;
+        for (int u = 0; u < 4; ++u) v[u] = (pg + 32 * u < pg1) ? __ldg(bt + pg + 32 * u) : 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (v[u] < 0 || v[u] >= p.num_pages) bad = 1;
+        for (int u = 0; u < 4; ++u)
+          if (v[u] < 0 || v[u] >= p.num_pages) bad = 1;
+      }
     }
 #pragma unroll
     for (int k = 0; k < kMaxTreeNodes / 32; ++k) {
@@ -681,11 +700,13 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
     const int node = (g.mp * kAttnQTiles + qt) * nodes_per_tile + r / p.group;
     const int head = g.kvh * p.group + (r % p.group);
     const bool row_valid = node < g.N;
-    if (static_cast<long long>(g.ke) * kBN > g.P && !build_ancestors(s, p, g)) ok = false;
+    // the segment reads a tile with tree keys (tiles P / kBN .. kt - 1) iff its rotated range reaches P / kBN
+    if (g.tile(g.kb) + (g.ke - g.kb) > g.P / kBN && !build_ancestors(s, p, g)) ok = false;
     const uint32_t* anc = &s.anc[row_valid ? node : 0][0];
     float m_use = -INFINITY, l = 0.f;
     for (int t = g.kb; t < g.ke; ++t, ++it) {
-      const bool tree_tile = (t + 1) * kBN > g.P;
+      const int kv = g.tile(t);
+      const bool tree_tile = (kv + 1) * kBN > g.P;
       if (!ok) continue;
       if (!warp_wait(&s.bar_sfull[qt], it & 1, abort)) {
         ok = false;
@@ -701,7 +722,7 @@ __device__ void softmax_epilogue(Smem& s, const AttnParams& p, SegIter iter, uin
       uint32_t vis[4];
 #pragma unroll
       for (int w = 0; w < 4; ++w)
-        vis[w] = tree_tile ? vis_word(t * kBN + 32 * w, g.P, g.N, row_valid, anc) : 0xffffffffu;
+        vis[w] = tree_tile ? vis_word(kv * kBN + 32 * w, g.P, g.N, row_valid, anc) : 0xffffffffu;
       tmem_ld_wait();
       tmem_ld32(lane_base + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
       tmem_ld32(lane_base + s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
