@@ -57,7 +57,11 @@ ATTN_SOURCES = ("tree_verify_attention_jf_b200/csrc/tree_attention.cu", "tree_ve
 # DRAM traffic of one tree_attention_kernel launch per workload (dram__bytes_read.sum + dram__bytes_write.sum of an
 # ncu capture of that workload), valid only for the kernel sources it was taken on: the roofline reports null once
 # any of them has changed.  Keys: bench workloads and legs.
-ATTN_TRAFFIC = {}
+ATTN_TRAFFIC = {
+    "qwen3_30b_a3b": dict(bytes=331_912_960 + 23_543_808, source_sha256="bba64c95b12d7e38c9e95397c5f832efa84e18ce1a5513905a4c3b9dccc39975"),
+    "qwen3_8b": dict(bytes=20_043_776 + 18_432, source_sha256="bba64c95b12d7e38c9e95397c5f832efa84e18ce1a5513905a4c3b9dccc39975"),
+    "serving": dict(bytes=298_771_968 + 18_972_160, source_sha256="bba64c95b12d7e38c9e95397c5f832efa84e18ce1a5513905a4c3b9dccc39975"),
+}
 
 
 def peaks():
@@ -119,8 +123,9 @@ HBM_BOUND = {"serving"}
 
 
 def roofline(workload, tflops, gbs, pk, flops, nbytes):
-    common = {"kernel": "jf_tree_attention (tree_attention_kernel + combine_kernel)",
-              "traffic": attention_traffic(workload), "algorithmic_flops": flops, "algorithmic_bytes": nbytes}
+    common = {"kernel": "jf_tree_attention: tree_attention_kernel then combine_kernel, timed together",
+              "traffic": attention_traffic(workload), "traffic_scope": "one tree_attention_kernel launch",
+              "algorithmic_flops": flops, "algorithmic_bytes": nbytes}
     if workload in HBM_BOUND:
         return dict(common, bound="hbm", achieved=gbs, peak=pk["hbm"], unit="GB/s", frac=gbs / pk["hbm"],
                     peak_source=pk["src"] + " HBM copy", tensor_achieved_tflops=tflops,

@@ -137,14 +137,24 @@ def test_qwen3_30b_exact_mask_probe():
 
 
 def test_workspace_reuse_and_determinism():
+    """One workspace, never initialised, serves calls with different splits in turn (the Qwen3-8B workload cuts
+    each unit over about five CTAs, the serving workload over two): what one call leaves there never leaks into
+    the next, and a repeated call gives the same bits (the merge order is fixed)."""
     inp = workloads.attention_workload("qwen3_8b")
+    srv = workloads.attention_workload("serving")
     ws = api.AttentionWorkspace(torch.device("cuda"))
     ws.buf.fill_(0x5A)  # the workspace needs no initialisation
-    d = to_dev(inp)
+    d, ds = to_dev(inp), to_dev(srv)
     a, la = run_attention(inp, ws=ws, dev=d)
+    s1, ls1 = run_attention(srv, ws=ws, dev=ds)
     b, lb = run_attention(inp, ws=ws, dev=d)
+    s2, ls2 = run_attention(srv, ws=ws, dev=ds)
     np.testing.assert_array_equal(a, b)
     np.testing.assert_array_equal(la, lb)
+    np.testing.assert_array_equal(s1, s2)
+    np.testing.assert_array_equal(ls1, ls2)
+    ref, lse_ref = tree_attention_inputs(inp)
+    compare(b, ref, lb, lse_ref)
 
 
 def test_cuda_graph_replay_matches_eager():
