@@ -1,7 +1,9 @@
 """The float64 exp used by the draft-logit row sums, checked on the host against math.exp (an
 independent libm) over the argument range the kernel sees, including the cutoff, and its table of
-2^(j/32) against exact decimal arithmetic.  The bound is 1e-14 relative: the row sums only need to keep
-the tree's float64 keys within far less than the 1e-9 decision margins the build tests guard."""
+2^(j/128) against exact decimal arithmetic.  The bound is 1e-14 relative: the row sums only need to keep
+the tree's float64 keys within far less than the 1e-9 decision margins the build tests guard.  At and below
+the cutoff (-709, where 2^k reaches 2^-1023) the result is a subnormal below 2.3e-308 rather than 0: next to the
+row maximum's exact 1 such a term changes no double-precision sum."""
 import math
 import os
 import shutil
@@ -40,8 +42,12 @@ def test_within_1e14_relative(exe):
 
 
 def test_cutoff_and_specials(exe):
-    got = run(exe, [-708.5, -1e6, float("-inf"), 0.0])
-    assert got[0] == 0.0 and got[1] == 0.0 and got[2] == 0.0 and got[3] == 1.0
+    got = run(exe, [-709.5, -1e6, float("-inf"), float("nan"), 0.0, -708.0])
+    assert all(0.0 <= g < 2.3e-308 for g in got[:4]), got[:4]
+    assert got[4] == 1.0
+    assert abs(got[5] - math.exp(-708.0)) <= 1e-14 * math.exp(-708.0)
+    # next to a row maximum's 1, a term at the cutoff leaves the sum unchanged
+    assert 1.0 + got[0] == 1.0
 
 
 def test_table_is_correctly_rounded(exe):
@@ -49,9 +55,9 @@ def test_table_is_correctly_rounded(exe):
     getcontext().prec = 60
     res = subprocess.run([exe, "table"], capture_output=True, text=True, check=True)
     tab = [float.fromhex(v) for v in res.stdout.split()]
-    assert len(tab) == 32
+    assert len(tab) == 128
     for j, d in enumerate(tab):
-        exact = Decimal(2) ** (Decimal(j) / Decimal(32))
+        exact = Decimal(2) ** (Decimal(j) / Decimal(128))
         err = abs(Decimal(d) - exact)
         # no neighbouring double is closer
         assert err <= abs(Decimal(math.nextafter(d, 0.0)) - exact), j

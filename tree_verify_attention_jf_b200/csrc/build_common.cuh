@@ -13,7 +13,7 @@ namespace jf {
 namespace build {
 
 // 2^(j/32) for the float64 exp (each translation unit keeps its own copy)
-static __device__ const double g_exp2_frac32[32] = JF_EXP2_FRAC32;
+static __device__ const double g_exp2_frac128[128] = JF_EXP2_FRAC128;
 
 constexpr int kThreads = 256;
 constexpr int kPerThread = kStatsChunk / kThreads;  // 16

@@ -44,14 +44,14 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ float s_max[kThreads / 32];
   __shared__ double s_sum[kThreads / 32];
   __shared__ Cand s_top[kThreads / 32][K];
-  __shared__ double s_tab[32];
+  __shared__ double s_tab[128];
   const int chunk = blockIdx.x, row = blockIdx.y;
   const int b = row / max_depth, d = row - b * max_depth;
   const float* x = logits + (static_cast<long long>(b) * depths + d) * vocab;
   const int lo = chunk * kStatsChunk;
   const int n = min(kStatsChunk, vocab - lo);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid < 32) s_tab[tid] = g_exp2_frac32[tid];  // visible after the barrier below
+  if (tid < 128) s_tab[tid] = g_exp2_frac128[tid];  // visible after the barrier below
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the logits' producer has completed
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (lim_nodes != nullptr) {
@@ -94,15 +94,23 @@ __global__ void __launch_bounds__(kThreads)
   Cand t[K];
 #pragma unroll
   for (int i = 0; i < K; ++i) t[i] = Cand{-INFINITY, INT_MAX};
+  if (n == kStatsChunk) {  // full chunk: no index checks
 #pragma unroll
-  for (int j = 0; j < kPerThread; ++j) {
-    const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
-    if (i < n) sum += exp_nonpos_f64(static_cast<double>(v[j]) - md, s_tab);
-  }
+    for (int j = 0; j < kPerThread; ++j) sum += exp_nonpos_f64(static_cast<double>(v[j]) - md, s_tab);
 #pragma unroll
-  for (int j = 0; j < kPerThread; ++j) {
-    const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
-    if (i < n && v[j] >= tau) insert_k<K>(t, Cand{v[j], lo + i});
+    for (int j = 0; j < kPerThread; ++j)
+      if (v[j] >= tau) insert_k<K>(t, Cand{v[j], lo + (j / 4) * kThreads * 4 + tid * 4 + (j & 3)});
+  } else {
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+      const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
+      if (i < n) sum += exp_nonpos_f64(static_cast<double>(v[j]) - md, s_tab);
+    }
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+      const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
+      if (i < n && v[j] >= tau) insert_k<K>(t, Cand{v[j], lo + i});
+    }
   }
   sum = warp_sum_d(sum);
   warp_merge_k<K>(t, 32);
@@ -136,7 +144,7 @@ __global__ void __launch_bounds__(kThreads)
 // Kernel 2: merge + best-first expansion.  grid = batch, block = 256
 // ------------------------------------------------------------------------------------------------
 struct ExpandSmem {
-  double tab[32];                       // 2^(j/32) for exp_nonpos_f64
+  double tab[128];                      // 2^(j/128) for exp_nonpos_f64
   double lp[kMaxDepths + 1][kMaxTopk];  // lp[d][r], d = 1..max_depth
   int tok[kMaxDepths + 1][kMaxTopk];
   double key[kMaxBudget];  // sequential fallback: node keys
@@ -287,7 +295,7 @@ __global__ void __launch_bounds__(kExpandThreads)
   SelectSmem& q = *reinterpret_cast<SelectSmem*>(dyn);
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid < 32) s.tab[tid] = g_exp2_frac32[tid];
+  if (tid < 128) s.tab[tid] = g_exp2_frac128[tid];
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the row statistics are complete
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int root_tok = tid == 0 ? root_tokens[b] : 0;  // in flight while the partials are merged

@@ -28,7 +28,7 @@ constexpr int kThreads = 512;
 constexpr int kPool = kMaxFrontierBudget * kMaxTopk;  // candidates of one sequence at most (2048)
 
 struct Smem {  // 44 KB: fits the static shared-memory limit
-  double tab[32];
+  double tab[128];
   double key[kMaxFrontierBudget];                // float64 key of every node
   double lp[kMaxFrontierBudget][kMaxTopk];       // candidate log-probabilities (their tokens stay in global memory)
   int depth[kMaxFrontierBudget];
@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ Smem s;
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid < 32) s.tab[tid] = build::g_exp2_frac32[tid];
+  if (tid < 128) s.tab[tid] = build::g_exp2_frac128[tid];
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the row statistics are complete
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long nb = static_cast<long long>(b) * budget;
