@@ -12,7 +12,7 @@
 namespace jf {
 namespace build {
 
-// 2^(j/32) for the float64 exp (each translation unit keeps its own copy)
+// 2^(j/128) for the float64 exp (each translation unit keeps its own copy)
 static __device__ const double g_exp2_frac128[128] = JF_EXP2_FRAC128;
 
 constexpr int kThreads = 256;
@@ -119,7 +119,7 @@ __device__ __forceinline__ double key_of_ord(unsigned long long o) {
 
 // One warp merges the chunk partials of one logits row: returns its natural-log LSE (the max, then the float64
 // sum of every chunk's sum scaled by exp(chunk max - max)) and leaves the row's best K by (logit desc, id asc)
-// in t on every lane.  tab: the 2^(j/32) table in shared memory.
+// in t on every lane.  tab: the 2^(j/128) table in shared memory.
 template <int K>
 __device__ __forceinline__ double warp_merge_row(const RowPartial* rp, int nchunks, int lane, const double* tab,
                                                  Cand (&t)[K]) {
