@@ -136,6 +136,33 @@ def test_qwen3_30b_exact_mask_probe():
     np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-4)
 
 
+def test_max_batch_ragged_with_empty_sequences():
+    """The largest batch the call takes (1024 sequences) with ragged trees of 0..8 nodes, about a quarter of the
+    sequences empty, over prefixes of 0..300 tokens in one interleaved page pool, g = 4: every row against the
+    oracle."""
+    rng = np.random.default_rng(31)
+    B = 1024
+    ns = rng.integers(0, 9, size=B)
+    ns[rng.random(B) < 0.25] = 0
+    prefix = rng.integers(0, 301, size=B)
+    parents = [synth.uniform_parent_tree(rng, int(n), 4) for n in ns]
+    inp = synth.attention_inputs(32, 8, 2, [int(p) for p in prefix], parents, interleave=True)
+    assert (ns == 0).sum() > 200 and inp.q.shape[0] == ns.sum()
+    out, lse = run_attention(inp)
+    ref, lse_ref = tree_attention_inputs(inp)
+    compare(out, ref, lse, lse_ref)
+
+
+def test_one_unit_cut_over_every_cta():
+    """One sequence, one kv head with g = 4 and 16 nodes (a single unit of 64 rows) over a 131072-token prefix: the
+    unit's 1025 kv tiles are split over every CTA, and the combine merges one segment from each of them."""
+    rng = np.random.default_rng(33)
+    inp = synth.attention_inputs(34, 4, 1, [131072], [synth.bushy_tree(rng, 16)])
+    out, lse = run_attention(inp)
+    ref, lse_ref = tree_attention_inputs(inp)
+    compare(out, ref, lse, lse_ref)
+
+
 def test_workspace_reuse_and_determinism():
     """One workspace, never initialised, serves calls with different splits in turn (the Qwen3-8B workload cuts
     each unit over about five CTAs, the serving workload over two): what one call leaves there never leaks into

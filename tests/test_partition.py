@@ -73,6 +73,7 @@ def segments(prefix, nodes, hkv, group, grid):
     (list(np.random.default_rng(0).integers(1024, 8193, 16)), [64] * 16, 8, 4, 148),
     ([0, 5, 300, 17], [3, 0, 256, 1], 2, 2, 7),
     ([10] * 50, [1] * 50, 1, 1, 148),
+    ([131072], [16], 1, 4, 148),  # one unit cut over every CTA
 ])
 def test_cover_exactly_once(prefix, nodes, hkv, group, grid):
     segs, W, G = segments(prefix, nodes, hkv, group, grid)
