@@ -102,6 +102,17 @@ def test_qwen3_8b_shape_and_scales():
     compare(out, ref, lse, lse_ref)
 
 
+def test_qwen3_30b_whole_workload():
+    """Every row of the Qwen3-30B-A3B workload over 8-bit caches (4 sequences x 256 nodes x 32 q heads, 32768-token
+    prefixes, g = 8): every unit is cut between several CTAs, so the conversion, the split partials and their
+    merge all run at full length."""
+    inp = workloads.attention_workload("qwen3_30b_a3b")
+    kc, vc = codes_of(inp)
+    out, lse = run_fp8(inp, kc, vc)
+    ref, lse_ref = reference(inp, kc, vc)
+    compare(out, ref, lse, lse_ref)
+
+
 def test_nan_codes_in_unused_slots_do_not_leak():
     inp = synth.attention_inputs(971, 4, 1, [20], [synth.uniform_parent_tree(np.random.default_rng(9), 10, 5)])
     kc, vc = codes_of(inp)
