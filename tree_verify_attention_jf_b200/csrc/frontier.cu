@@ -27,7 +27,7 @@ using build::Cand;
 constexpr int kThreads = 512;
 constexpr int kPool = kMaxFrontierBudget * kMaxTopk;  // candidates of one sequence at most (2048)
 
-struct Smem {  // 44 KB: fits the static shared-memory limit
+struct Smem {  // 45 KB: fits the static shared-memory limit (48 KB)
   double tab[128];
   double key[kMaxFrontierBudget];                // float64 key of every node
   double lp[kMaxFrontierBudget][kMaxTopk];       // candidate log-probabilities (their tokens stay in global memory)

@@ -90,7 +90,7 @@ JF_HD double exp_nonpos_f64(double x, const double* tab) {
   // 2^k * 2^(j/128): the entry's exponent field (1023) plus k stays in [0, 1023]
   double s;
 #if defined(__CUDA_ARCH__)
-  s = __hiloint2double(__double2hiint(tab[j]) + (k << 20), __double2loint(tab[j]));
+  s = __hiloint2double(__double2hiint(tab[j]) + k * (1 << 20), __double2loint(tab[j]));
 #else
   uint64_t bits;
   std::memcpy(&bits, &tab[j], sizeof(bits));
