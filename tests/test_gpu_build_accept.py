@@ -65,6 +65,23 @@ def test_build_ties_across_chunks():
     assert (got["depth"] == 2).sum() == 2 * 16
 
 
+@pytest.mark.parametrize("hot", [40, 300, 700])
+def test_build_many_tied_maxima_per_chunk(hot):
+    # `hot` entries of every 4096-entry chunk share the row's largest logit, so that tens to hundreds of
+    # elements per chunk pass the per-warp filter (700 is more than a chunk's candidate list holds); the
+    # lowest ids among them must win
+    rng = np.random.default_rng(11 + hot)
+    V = 20000
+    x = rng.normal(0.0, 2.0, size=(2, 4, V)).astype(np.float32)
+    for c0 in range(0, V, 4096):
+        n = min(4096, V - c0)
+        for b in range(2):
+            for d in range(4):
+                idx = c0 + rng.choice(n, size=min(hot, n), replace=False)
+                x[b, d, idx] = 12.0 + d
+    check_build(x, np.array([1, 2]), 4, 60, 4, margin_guard=False)
+
+
 def gpu_accept(tok, par, tgt, max_depth):
     res = api.accept(torch.from_numpy(np.ascontiguousarray(tok, dtype=np.int32)).cuda(),
                      torch.from_numpy(np.ascontiguousarray(par, dtype=np.int32)).cuda(),

@@ -17,6 +17,10 @@ static __device__ const double g_exp2_frac128[128] = JF_EXP2_FRAC128;
 
 constexpr int kThreads = 256;
 constexpr int kPerThread = kStatsChunk / kThreads;  // 16
+constexpr int kCandCap = 512;  // row-statistics candidate list per CTA (4 KB)
+// row-statistics CTAs resident per SM: 8 (32 registers a thread) for lists of up to 4, 5 (48) for 8, which
+// would spill at 32
+constexpr int stats_ctas_per_sm(int K) { return K <= 4 ? 8 : 5; }
 constexpr int kSlots = kMaxDepths * kMaxTopk / 32;  // queue slots per lane (16)
 
 struct Cand {
@@ -93,13 +97,15 @@ __device__ __forceinline__ float warp_max_f(float x) {
 
 // A lower bound on the K-th largest of the warp's 32 values: K rounds of "take the warp max, drop every
 // lane that holds it".  Ties are dropped together, so the result is the K-th largest distinct value
-// (or -inf if there are fewer), which never exceeds the K-th largest counted with multiplicity.
+// (or -inf if there are fewer), which never exceeds the K-th largest counted with multiplicity.  The
+// first round's maximum (the warp max) is returned in mx.
 template <int K>
-__device__ __forceinline__ float warp_kth_bound(float x) {
+__device__ __forceinline__ float warp_kth_bound(float x, float& mx) {
   float m = -INFINITY;
 #pragma unroll
   for (int r = 0; r < K; ++r) {
     m = warp_max_f(x);
+    if (r == 0) mx = m;
     if (x == m) x = -INFINITY;
   }
   return m;

@@ -37,7 +37,7 @@ namespace build {
 // size: lim_nodes[b] - lim_begin[b] rows, 1 (the root's) for a tree that has no node yet, none for a tree that
 // already holds lim_budget nodes.
 template <int K>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, stats_ctas_per_sm(K))
     row_stats_kernel(const float* __restrict__ logits, int depths, int vocab, int max_depth,
                      RowPartial* __restrict__ out, const int32_t* __restrict__ lim_nodes,
                      const int32_t* __restrict__ lim_begin, int lim_budget) {
@@ -45,13 +45,16 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ double s_sum[kThreads / 32];
   __shared__ Cand s_top[kThreads / 32][K];
   __shared__ double s_tab[128];
+  __shared__ Cand s_cand[kCandCap];  // elements that pass their warp's top-K filter
+  __shared__ int s_cnt;
   const int chunk = blockIdx.x, row = blockIdx.y;
   const int b = row / max_depth, d = row - b * max_depth;
   const float* x = logits + (static_cast<long long>(b) * depths + d) * vocab;
   const int lo = chunk * kStatsChunk;
   const int n = min(kStatsChunk, vocab - lo);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid < 128) s_tab[tid] = g_exp2_frac128[tid];  // visible after the barrier below
+  const double tab_entry = g_exp2_frac128[tid & 127];  // stored once the chunk's loads are issued
+  if (tid == 0) s_cnt = 0;
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the logits' producer has completed
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (lim_nodes != nullptr) {
@@ -77,13 +80,14 @@ __global__ void __launch_bounds__(kThreads)
       v[j] = (i < n) ? __ldg(x + lo + i) : -INFINITY;
     }
   }
+  if (tid < 128) s_tab[tid] = tab_entry;  // visible after the barrier below
   float m_lane = -INFINITY;
 #pragma unroll
   for (int j = 0; j < kPerThread; ++j) m_lane = fmaxf(m_lane, v[j]);
   // Top-K filter: the K largest lane maxima are K distinct elements of the warp, so an element below
   // the K-th of them cannot be among the warp's (hence the chunk's) best K, whatever the tie-break.
-  const float tau = warp_kth_bound<K>(m_lane);
-  float m = warp_max_f(m_lane);
+  float m;  // the warp's max, then the chunk's
+  const float tau = warp_kth_bound<K>(m_lane, m);
   if (lane == 0) s_max[warp] = m;
   __syncthreads();
   m = s_max[0];
@@ -91,41 +95,64 @@ __global__ void __launch_bounds__(kThreads)
   for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, s_max[w]);
   const double md = static_cast<double>(m);
   double sum = 0.0;
-  Cand t[K];
-#pragma unroll
-  for (int i = 0; i < K; ++i) t[i] = Cand{-INFINITY, INT_MAX};
-  if (n == kStatsChunk) {  // full chunk: no index checks
+  const bool full = n == kStatsChunk;
+  if (full) {  // no index checks
 #pragma unroll
     for (int j = 0; j < kPerThread; ++j) sum += exp_nonpos_f64(static_cast<double>(v[j]) - md, s_tab);
-#pragma unroll
-    for (int j = 0; j < kPerThread; ++j)
-      if (v[j] >= tau) insert_k<K>(t, Cand{v[j], lo + (j / 4) * kThreads * 4 + tid * 4 + (j & 3)});
   } else {
 #pragma unroll
     for (int j = 0; j < kPerThread; ++j) {
       const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
       if (i < n) sum += exp_nonpos_f64(static_cast<double>(v[j]) - md, s_tab);
     }
+  }
+  // The few elements at or above the filter bound go to one shared list (typically K to 2K per warp);
+  // warp 0 selects the chunk's best K from it.  The best K under (logit desc, id asc) is unique, so the
+  // order of the list does not matter.
 #pragma unroll
-    for (int j = 0; j < kPerThread; ++j) {
-      const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
-      if (i < n && v[j] >= tau) insert_k<K>(t, Cand{v[j], lo + i});
+  for (int j = 0; j < kPerThread; ++j) {
+    const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
+    if (v[j] >= tau && (full || i < n)) {
+      const int pos = atomicAdd(&s_cnt, 1);
+      if (pos < kCandCap) s_cand[pos] = Cand{v[j], lo + i};
     }
   }
   sum = warp_sum_d(sum);
-  warp_merge_k<K>(t, 32);
-  if (lane == 0) {
-    s_sum[warp] = sum;
-#pragma unroll
-    for (int i = 0; i < K; ++i) s_top[warp][i] = t[i];
-  }
+  if (lane == 0) s_sum[warp] = sum;
   __syncthreads();
+  const int cnt = s_cnt;  // uniform over the CTA
+  Cand t[K];
+#pragma unroll
+  for (int i = 0; i < K; ++i) t[i] = Cand{-INFINITY, INT_MAX};
+  if (cnt > kCandCap) {
+    // list overflow (heavy ties under the bound): every warp merges its own elements, read again from
+    // memory, then warp 0 merges the warps' lists
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+      const int i = (j / 4) * kThreads * 4 + tid * 4 + (j & 3);
+      if (i < n) {
+        const float xi = __ldg(x + lo + i);
+        if (xi >= tau) insert_k<K>(t, Cand{xi, lo + i});
+      }
+    }
+    warp_merge_k<K>(t, 32);
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < K; ++i) s_top[warp][i] = t[i];
+    }
+    __syncthreads();
+  }
   if (warp == 0) {
     double ssum = (lane < kThreads / 32) ? s_sum[lane] : 0.0;
     ssum = warp_sum_d(ssum);
+    if (cnt > kCandCap) {
 #pragma unroll
-    for (int i = 0; i < K; ++i) t[i] = (lane < kThreads / 32) ? s_top[lane][i] : Cand{-INFINITY, INT_MAX};
-    warp_merge_k<K>(t, 8);
+      for (int i = 0; i < K; ++i) t[i] = (lane < kThreads / 32) ? s_top[lane][i] : Cand{-INFINITY, INT_MAX};
+      warp_merge_k<K>(t, 8);
+    } else {
+      for (int c = lane; c < cnt; c += 32) insert_k<K>(t, s_cand[c]);
+      warp_merge_k<K>(t, 32);
+    }
     if (lane == 0) {
       RowPartial& o = out[static_cast<long long>(row) * gridDim.x + chunk];
       o.sum = ssum;
