@@ -58,9 +58,9 @@ ATTN_SOURCES = ("tree_verify_attention_jf_b200/csrc/tree_attention.cu", "tree_ve
 # ncu capture of that workload), valid only for the kernel sources it was taken on: the roofline reports null once
 # any of them has changed.  Keys: bench workloads and legs.
 ATTN_TRAFFIC = {
-    "qwen3_30b_a3b": dict(bytes=331_912_960 + 23_543_808, source_sha256="bba64c95b12d7e38c9e95397c5f832efa84e18ce1a5513905a4c3b9dccc39975"),
-    "qwen3_8b": dict(bytes=20_043_776 + 18_432, source_sha256="bba64c95b12d7e38c9e95397c5f832efa84e18ce1a5513905a4c3b9dccc39975"),
-    "serving": dict(bytes=298_771_968 + 18_972_160, source_sha256="bba64c95b12d7e38c9e95397c5f832efa84e18ce1a5513905a4c3b9dccc39975"),
+    "qwen3_30b_a3b": dict(bytes=329_136_640 + 21_105_152, source_sha256="450ae8dfb4740ae7caef691319b2c4ef0d143c150fde992d2f737ad539945d9f"),
+    "qwen3_8b": dict(bytes=20_044_800 + 24_576, source_sha256="450ae8dfb4740ae7caef691319b2c4ef0d143c150fde992d2f737ad539945d9f"),
+    "serving": dict(bytes=298_685_696 + 17_516_032, source_sha256="450ae8dfb4740ae7caef691319b2c4ef0d143c150fde992d2f737ad539945d9f"),
 }
 
 

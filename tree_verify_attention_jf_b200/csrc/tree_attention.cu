@@ -230,10 +230,10 @@ __device__ void build_plan(Smem& s, const AttnParams& p) {
 // stage.  A warp converts 16 rows per step (4 chunks of 16 bytes per lane, all read before any is written): the
 // writes of a step land in rows [0, 16 KB) and on the 8-bit rows the same step has just read, so rows still to
 // be read are never overwritten.
-__device__ __forceinline__ void convert_stage_e4m3(uint8_t* stage, int lane) {
+__device__ __forceinline__ void convert_stage_e4m3_step(uint8_t* stage, int lane, int r0) {
   const int c = lane & 7;  // 16-byte chunk of the 8-bit row: dims [16 c, 16 c + 16)
   const int j0 = 2 * (c & 3);  // its f16 bytes are chunks j0, j0 + 1 of half c / 4
-  for (int r0 = 0; r0 < kBN; r0 += 16) {
+  {
     uint4 raw[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k)
@@ -259,6 +259,7 @@ __device__ __forceinline__ void convert_stage_e4m3(uint8_t* stage, int lane) {
     __syncwarp();
   }
 }
+constexpr int kConvSteps = kBN / 16;  // 16-row steps per stage
 
 // The Q tiles in place, bf16 -> f16, element by element (the swizzle does not matter).
 __device__ __forceinline__ void convert_q_bf16_f16(uint8_t* q, int bytes, int lane) {
@@ -277,8 +278,9 @@ __device__ __forceinline__ void convert_q_bf16_f16(uint8_t* q, int bytes, int la
 
 // ------------------------------------------------------------------------------------------------
 // Warps 0 and 2: K / V gathers (warp 0 also loads the Q tiles).  With an 8-bit cache each tile lands on a
-// barrier of its own; the warp converts it after issuing the next tile's copies and then arrives on the
-// full barrier the MMA warp waits on (the Q tiles likewise, after the segment's first K tile).
+// barrier of its own; while the warp waits for a stage to free it converts the landed tiles in order, 16 rows
+// at a time, and arrives on the full barrier the MMA warp waits on once a tile is done (the Q tiles are
+// converted right after the segment's first K tile is issued).
 // ------------------------------------------------------------------------------------------------
 template <bool kFp8>
 __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_v, const CUtensorMap* tm_q,
@@ -291,8 +293,8 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
   uint64_t* qland = kFp8 ? &s.bar_qland : &s.bar_qfull;
   Seg g;
   uint32_t it = 0, sidx = 0;
-  int pend_st = -1;  // 8-bit cache: a landed tile not yet converted (stage), its landing parity
-  uint32_t pend_ph = 0;
+  uint32_t cit = 0;  // 8-bit cache: tiles converted so far (tiles [cit, it) are issued and not yet converted)
+  int cstep = 0;     // next 16-row step of tile cit
   bool q_pend = false;
   // the latest phase this warp armed on each landing barrier (bit st of armed; its parity in armed_par), and on
   // the Q landing barrier: on an abort the warp waits for them, i.e. for every copy it issued
@@ -303,14 +305,32 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
       if (armed & (1u << st)) drain_wait(&land[st], (armed_par >> st) & 1u);
     if (q_armed) drain_wait(qland, q_par);
   };
-  auto convert_pending = [&]() -> bool {
-    if (!kFp8 || pend_st < 0) return true;
-    if (!warp_wait(&land[pend_st], pend_ph, abort)) return false;
-    convert_stage_e4m3(is_v ? s.v[pend_st] : s.k[pend_st], lane);
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&full[pend_st]);
-    pend_st = -1;
+  // One step of the oldest unconverted tile: 1 = done, 0 = nothing to convert or (block false) not landed yet,
+  // -1 = the landing wait ran out.  The tile's last step hands it to the MMA warp.
+  auto conv_step = [&](bool block) -> int {
+    if (!kFp8 || cit == it) return 0;
+    const int cst = cit % kStages;
+    const uint32_t cph = (cit / kStages) & 1;
+    if (cstep == 0) {
+      if (block) {
+        if (!warp_wait(&land[cst], cph, abort)) return -1;
+      } else if (!__all_sync(0xffffffffu, mbar_test_wait(&land[cst], cph))) {
+        return 0;
+      }
+    }
+    convert_stage_e4m3_step(is_v ? s.v[cst] : s.k[cst], lane, cstep * 16);
+    if (++cstep == kConvSteps) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[cst]);
+      cstep = 0;
+      ++cit;
+    }
+    return 1;
+  };
+  auto convert_all = [&]() -> bool {
+    while (cit != it)
+      if (conv_step(true) < 0) return false;
     return true;
   };
   const int nodes_per_tile = kBM / p.group;
@@ -333,9 +353,9 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
     };
     int ids_cur = batch_ids(g.kb);
     int ids_next = batch_ids(g.kb + 4);
-    // 8-bit cache: the previous segment's last tile is converted now -- the Q buffer frees only after that
-    // tile's QK has run
-    if (!convert_pending()) return unwind();
+    // 8-bit cache: the previous segment's last K tiles are converted now -- the Q buffer frees only after their
+    // QKs have run
+    if (!is_v && !convert_all()) return unwind();
     // the Q tiles go out while the page ids are on their way
     if (!is_v) {
       if (!warp_wait(&s.bar_qempty, (sidx & 1) ^ 1, abort)) return unwind();
@@ -363,7 +383,21 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
       if (lane >= (kFp8 ? 1 : 2) * kPagesPerTile) pid = -1;
       const uint32_t mask = __ballot_sync(0xffffffffu, pid >= 0);
       const uint32_t bytes = static_cast<uint32_t>(__popc(mask)) * (kPage * 128u);
-      if (!warp_wait(&empty[st], ph ^ 1, abort)) return unwind();
+      if (kFp8) {
+        // convert landed tiles step by step while the stage is still in use
+        const uint64_t t0 = globaltimer();
+        uint32_t spins = 0;
+        while (!__all_sync(0xffffffffu, mbar_test_wait(&empty[st], ph ^ 1))) {
+          const int r = conv_step(false);
+          if (r < 0) return unwind();
+          if (r == 0) {
+            __nanosleep(64);
+            if ((++spins & 31u) == 0 && (*abort || globaltimer() - t0 > kWaitLimitNs)) return unwind();
+          }
+        }
+      } else if (!warp_wait(&empty[st], ph ^ 1, abort)) {
+        return unwind();
+      }
       if (is_v && it == 0) {
         // The copy engine serves requests in order and the first S needs Q and K only: the kernel's
         // first V tile is queued behind the first K tile (bounded wait, like every other).
@@ -391,10 +425,7 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
         if (lane == 0) *reinterpret_cast<volatile int*>(&s.k_started) = 1;
       }
       if (kFp8) {
-        // convert the previous tile while this one is on its way, then (segment start) the Q tiles
-        if (!convert_pending()) return unwind();
-        pend_st = st;
-        pend_ph = ph;
+        // segment start: the Q tiles, while this K tile is on its way
         if (q_pend) {
           if (!warp_wait(&s.bar_qland, sidx & 1, abort)) return unwind();
           convert_q_bf16_f16(&s.q[0][0], kAttnQTiles * kTileBytes, lane);
@@ -407,7 +438,7 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
     }
     ++sidx;
   }
-  if (!convert_pending()) return unwind();
+  if (!convert_all()) return unwind();
 }
 
 // ------------------------------------------------------------------------------------------------
