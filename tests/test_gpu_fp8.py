@@ -113,6 +113,34 @@ def test_qwen3_30b_whole_workload():
     compare(out, ref, lse, lse_ref)
 
 
+def test_max_batch_ragged_with_empty_sequences():
+    """1024 sequences with ragged trees of 0..8 nodes (about a quarter empty) over prefixes of 0..300 tokens, g = 4:
+    every CTA runs many one- to three-tile segments, so landed tiles are still being converted when the next
+    segment's Q tiles go out."""
+    rng = np.random.default_rng(41)
+    B = 1024
+    ns = rng.integers(0, 9, size=B)
+    ns[rng.random(B) < 0.25] = 0
+    prefix = rng.integers(0, 301, size=B)
+    parents = [synth.uniform_parent_tree(rng, int(n), 4) for n in ns]
+    inp = synth.attention_inputs(42, 8, 2, [int(p) for p in prefix], parents, interleave=True)
+    kc, vc = codes_of(inp)
+    out, lse = run_fp8(inp, kc, vc)
+    ref, lse_ref = reference(inp, kc, vc)
+    compare(out, ref, lse, lse_ref)
+
+
+def test_one_unit_cut_over_every_cta():
+    """One unit (16 nodes, g = 4) over a 131072-token prefix: its 1025 kv tiles are split over every CTA, and
+    each CTA's segment converts a handful of tiles and writes a partial."""
+    rng = np.random.default_rng(43)
+    inp = synth.attention_inputs(44, 4, 1, [131072], [synth.bushy_tree(rng, 16)])
+    kc, vc = codes_of(inp)
+    out, lse = run_fp8(inp, kc, vc)
+    ref, lse_ref = reference(inp, kc, vc)
+    compare(out, ref, lse, lse_ref)
+
+
 def test_nan_codes_in_unused_slots_do_not_leak():
     inp = synth.attention_inputs(971, 4, 1, [20], [synth.uniform_parent_tree(np.random.default_rng(9), 10, 5)])
     kc, vc = codes_of(inp)
