@@ -58,8 +58,8 @@ __global__ void __launch_bounds__(kThreads, stats_ctas_per_sm(K))
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the logits' producer has completed
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (lim_nodes != nullptr) {
-    const int n = lim_nodes[b];
-    const int rows = (n == 0) ? 1 : (n >= lim_budget ? 0 : n - lim_begin[b]);
+    const int nodes = lim_nodes[b];
+    const int rows = (nodes == 0) ? 1 : (nodes >= lim_budget ? 0 : nodes - lim_begin[b]);
     if (d >= rows) return;  // uniform over the CTA: a row outside the frontier is never read
   }
   float v[kPerThread];
