@@ -227,37 +227,35 @@ __device__ void build_plan(Smem& s, const AttnParams& p) {
 // ------------------------------------------------------------------------------------------------
 // One K or V stage: the copy put the tile's 8-bit rows (128 keys x 128 dims, one 128-byte row per key) in the
 // stage's upper 16 KB; they become f16 in the 128-byte-swizzled [half][128 keys][64 dims] layout of the whole
-// stage.  A warp converts 16 rows per step (4 chunks of 16 bytes per lane, all read before any is written): the
-// writes of a step land in rows [0, 16 KB) and on the 8-bit rows the same step has just read, so rows still to
-// be read are never overwritten.
+// stage.  A warp converts 16 rows [r0, r0 + 16) per step (4 chunks of 16 bytes per lane, all read before any is
+// written), the steps in order r0 = 0, 16, ..., 112: the writes of a step land in rows [0, 16 KB) and on the 8-bit
+// rows the same step has just read, so rows still to be read are never overwritten.
 __device__ __forceinline__ void convert_stage_e4m3_step(uint8_t* stage, int lane, int r0) {
   const int c = lane & 7;  // 16-byte chunk of the 8-bit row: dims [16 c, 16 c + 16)
   const int j0 = 2 * (c & 3);  // its f16 bytes are chunks j0, j0 + 1 of half c / 4
-  {
-    uint4 raw[4];
+  uint4 raw[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      raw[k] = *reinterpret_cast<const uint4*>(stage + kHalfBytes + (r0 + (lane >> 3) + 4 * k) * 128 + c * 16);
-    __syncwarp();
+  for (int k = 0; k < 4; ++k)
+    raw[k] = *reinterpret_cast<const uint4*>(stage + kHalfBytes + (r0 + (lane >> 3) + 4 * k) * 128 + c * 16);
+  __syncwarp();
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int row = r0 + (lane >> 3) + 4 * k;
-      const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
-      uint32_t hv[8];
+  for (int k = 0; k < 4; ++k) {
+    const int row = r0 + (lane >> 3) + 4 * k;
+    const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+    uint32_t hv[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const __half2_raw lo =
-            __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xffffu), __NV_E4M3);
-        const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
-        hv[2 * i] = static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16);
-        hv[2 * i + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
-      }
-      uint8_t* base = stage + (c >> 2) * kHalfBytes + row * 128;
-      *reinterpret_cast<uint4*>(base + ((j0 ^ (row & 7)) * 16)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-      *reinterpret_cast<uint4*>(base + (((j0 + 1) ^ (row & 7)) * 16)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+    for (int i = 0; i < 4; ++i) {
+      const __half2_raw lo =
+          __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xffffu), __NV_E4M3);
+      const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
+      hv[2 * i] = static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16);
+      hv[2 * i + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
     }
-    __syncwarp();
+    uint8_t* base = stage + (c >> 2) * kHalfBytes + row * 128;
+    *reinterpret_cast<uint4*>(base + ((j0 ^ (row & 7)) * 16)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    *reinterpret_cast<uint4*>(base + (((j0 + 1) ^ (row & 7)) * 16)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
   }
+  __syncwarp();
 }
 constexpr int kConvSteps = kBN / 16;  // 16-row steps per stage
 
@@ -391,6 +389,8 @@ __device__ void kv_producer(Smem& s, const AttnParams& p, SegIter iter, bool is_
           const int r = conv_step(false);
           if (r < 0) return unwind();
           if (r == 0) {
+            // a short sleep hands the SMSP's issue slots to the softmax warps; a landing or a free stage is
+            // still seen within a fraction of a conversion step
             __nanosleep(64);
             if ((++spins & 31u) == 0 && (*abort || globaltimer() - t0 > kWaitLimitNs)) return unwind();
           }
