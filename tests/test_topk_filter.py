@@ -38,3 +38,39 @@ def test_filter_keeps_the_best_k(K, kind):
         tau = kth_bound(v.max(axis=1), K)
         keep = v >= tau
         assert best_k(v[keep], ids[keep], K) == best_k(v.ravel(), ids.ravel(), K)
+
+
+@pytest.mark.parametrize("K", [1, 2, 4, 8])
+def test_chunk_candidate_list(K):
+    """One 4096-entry chunk = 8 warps x 32 lanes x 16 entries: the elements that pass their own warp's bound form
+    one list, and the chunk's best K taken from that list is the chunk's best K.  On logits with a spread like a
+    draft head's (normal, or a peaked head over a flat tail) the list stays far below its 512 entries; a chunk of
+    a few distinct values (heavy ties) overflows it, which the kernel handles by merging per warp instead."""
+    CAP = 512
+    rng = np.random.default_rng(100 + K)
+    ids = np.array([[[(j // 4) * 1024 + (w * 32 + l) * 4 + (j & 3) for j in range(16)] for l in range(32)]
+                    for w in range(8)])
+    assert sorted(ids.ravel().tolist()) == list(range(4096))
+    longest = 0
+    for trial in range(150):
+        if trial % 3 == 0:
+            v = rng.standard_normal((8, 32, 16)).astype(np.float32)
+        elif trial % 3 == 1:
+            v = (rng.standard_normal((8, 32, 16)) * 0.1).astype(np.float32)
+            hot = rng.integers(0, 4096, 5)
+            v.reshape(-1)[hot] += rng.uniform(5, 10, 5).astype(np.float32)
+        else:
+            v = rng.gumbel(size=(8, 32, 16)).astype(np.float32)
+        cand_v, cand_i = [], []
+        for w in range(8):
+            tau = kth_bound(v[w].max(axis=1), K)
+            keep = v[w] >= tau
+            cand_v.append(v[w][keep])
+            cand_i.append(ids[w][keep])
+        cv, ci = np.concatenate(cand_v), np.concatenate(cand_i)
+        longest = max(longest, cv.size)
+        assert best_k(cv, ci, K) == best_k(v.ravel(), ids.ravel(), K)
+    assert longest < CAP // 4, longest
+    ties = rng.integers(0, 3, size=(8, 32, 16)).astype(np.float32)
+    n = sum(int((ties[w] >= kth_bound(ties[w].max(axis=1), K)).sum()) for w in range(8))
+    assert n > CAP  # the overflow path is the one heavy ties take
