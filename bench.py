@@ -58,9 +58,9 @@ ATTN_SOURCES = ("tree_verify_attention_jf_b200/csrc/tree_attention.cu", "tree_ve
 # ncu capture of that workload), valid only for the kernel sources it was taken on: the roofline reports null once
 # any of them has changed.  Keys: bench workloads and legs.
 ATTN_TRAFFIC = {
-    "qwen3_30b_a3b": dict(bytes=330_297_344 + 21_158_656, source_sha256="9e6478b345a9ea9e7d02d0b5fd4f2e7bb51f7199cc2c47f76c5e6962da477f46"),
-    "qwen3_8b": dict(bytes=20_043_776 + 28_672, source_sha256="9e6478b345a9ea9e7d02d0b5fd4f2e7bb51f7199cc2c47f76c5e6962da477f46"),
-    "serving": dict(bytes=298_674_176 + 17_058_304, source_sha256="9e6478b345a9ea9e7d02d0b5fd4f2e7bb51f7199cc2c47f76c5e6962da477f46"),
+    "qwen3_30b_a3b": dict(bytes=331_310_080 + 21_271_040, source_sha256="c77f7b6b23b3b21b197d8eb90cb4a50a49a0de2978c769ccc8fa8f3d5d042b79"),
+    "qwen3_8b": dict(bytes=20_044_032 + 33_792, source_sha256="c77f7b6b23b3b21b197d8eb90cb4a50a49a0de2978c769ccc8fa8f3d5d042b79"),
+    "serving": dict(bytes=298_682_624 + 17_449_216, source_sha256="c77f7b6b23b3b21b197d8eb90cb4a50a49a0de2978c769ccc8fa8f3d5d042b79"),
 }
 
 

@@ -986,9 +986,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Register split (the launch gives every thread 168): the copy/MMA/metadata warpgroup runs on 80,
   // which lets the two softmax warpgroups hold a whole 128-column row of S in registers (208).
-  // 128 * 80 + 256 * 208 = 63488 <= 384 * 168 = 64512 (the launch's register pool).
+  // 128 * 80 + 256 * 208 = 63488 <= 384 * 168 = 64512 (the launch's register pool).  With an 8-bit cache
+  // the copy warps also convert every tile, which spills at 80: there the split is 104 / 200
+  // (128 * 104 + 256 * 200 = 64512).
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
+    if (kFp8) asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
+    else asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
     if (warp == 0 || warp == 2) {
       kv_producer<kFp8>(s, p, iter, warp == 2, &tm_q, warp == 2 ? &tm_v : &tm_k);
     } else if (warp == 1) {
@@ -997,7 +1000,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       metadata(s, p, iter);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
+    if (kFp8) asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
+    else asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
     softmax_epilogue<kFp8>(s, p, iter, tmem, warp < 8 ? 0 : 1);
   }
   tc_fence_before();
